@@ -1,0 +1,266 @@
+"""Oracle for the fused ShortConv K/V step -- TEST INFRASTRUCTURE ONLY.
+
+A thin ctypes/numpy front end over ``sconv_kv_oracle.c`` (plain double
+precision loops, one step of the method per function; see that file's header
+for the passages each step follows and the readings taken where the pages are
+silent).  Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg may import this package.  It never touches the GPU and
+shares nothing with the CUDA library.
+
+Arrays are numpy: bf16 tensors travel as their uint16 bit patterns.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+ERRORS = {
+    0: "ok",
+    -1: "bad argument",
+    -2: "slot out of range",
+    -3: "duplicate slot",
+    -4: "state index out of range",
+    -5: "cu_seqlens is not a partition of the tokens",
+    -6: "out of memory",
+}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code):
+        super().__init__(f"oracle returned {code}: {ERRORS.get(code, '?')}")
+        self.code = code
+
+
+def load(path=None):
+    """Load (building first if needed) the oracle library."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    if path is None:
+        if _build.needs_build():
+            _build.build()
+        path = _build.LIB
+    lib = ctypes.CDLL(path)
+    lib.oracle_conv.argtypes = [_u16p, _i64, _i64, _u16p, _i64, _u16p, _int,
+                                _int, _f64p]
+    lib.oracle_conv.restype = None
+    lib.oracle_rmsnorm.argtypes = [_f64p, _i64, _int, _int, _f32p,
+                                   ctypes.c_double, _f64p]
+    lib.oracle_rmsnorm.restype = None
+    lib.oracle_scatter.argtypes = [_f64p, _i64, _int, _int, _i64p, _i64, _i64,
+                                   _i64, _i64, _i64, _u16p]
+    lib.oracle_scatter.restype = _int
+    lib.oracle_state_update.argtypes = [_u16p, _i64, _i64, _u16p, _i64, _int,
+                                        _int]
+    lib.oracle_state_update.restype = None
+    common_tail = [_u16p, _i32p, _i64, _i64p, _u16p, _u16p, _i64, _i64, _i64,
+                   _i64, _i64, _f64p, _f64p]
+    lib.oracle_prefill_varlen.argtypes = (
+        [_u16p, _u16p, _i64, _i64, _i32p, _int, _u16p, _u16p, _f32p, _f32p,
+         ctypes.c_double, _int, _int, _int] + common_tail)
+    lib.oracle_prefill_varlen.restype = _int
+    lib.oracle_decode.argtypes = (
+        [_u16p, _u16p, _i64, _int, _u16p, _u16p, _f32p, _f32p,
+         ctypes.c_double, _int, _int, _int] + common_tail)
+    lib.oracle_decode.restype = _int
+    lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_to_double.restype = ctypes.c_double
+    lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+    lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_round_bf16_array.argtypes = [_f64p, _i64, _u16p]
+    lib.oracle_round_bf16_array.restype = None
+    if path == _build.LIB:
+        _lib = lib
+    return lib
+
+
+def _p(a, ptype):
+    if a is None:
+        return ctypes.cast(None, ptype)
+    assert a.flags["C_CONTIGUOUS"], "oracle wants C-contiguous arrays"
+    return a.ctypes.data_as(ptype)
+
+
+def _u16(a):
+    a = np.asarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected uint16 bf16 bit patterns, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
+# ---------------------------------------------------------------- bf16 bits
+
+def bf16_bits_to_f64(bits):
+    """Exact widening of bf16 bit patterns to float64."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_to_bf16_bits(x, lib=None):
+    """Round float64 values to bf16 (nearest, ties to even), one rounding."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib.oracle_round_bf16_array(_p(x, _f64p), x.size, _p(out, _u16p))
+    return out
+
+
+# ---------------------------------------------------------------- stages
+
+def conv(x, state, w, lib=None):
+    """Step a1+a2 for one tensor of one sequence.
+
+    x: uint16 [L, C]; state: uint16 [W-1, C] (old rows, oldest first);
+    w: uint16 [W, C].  Returns float64 y [L, C].
+    """
+    lib = lib or load()
+    x, w = _u16(x), _u16(w)
+    W, C = w.shape
+    L = x.shape[0]
+    state = _u16(state) if W > 1 else np.zeros((1, C), np.uint16)
+    y = np.empty((L, C), np.float64)
+    lib.oracle_conv(_p(x, _u16p), C, L, _p(state, _u16p), C, _p(w, _u16p),
+                    W, C, _p(y, _f64p))
+    return y
+
+
+def rmsnorm(y, num_heads, gamma, eps, lib=None):
+    """Step a3: y float64 [L, H*D] -> z float64 [L, H*D]."""
+    lib = lib or load()
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    gamma = np.ascontiguousarray(gamma, dtype=np.float32)
+    L = y.shape[0]
+    D = gamma.shape[0]
+    z = np.empty_like(y)
+    lib.oracle_rmsnorm(_p(y, _f64p), L, num_heads, D, _p(gamma, _f32p),
+                       float(eps), _p(z, _f64p))
+    return z
+
+
+def scatter(z, num_heads, D, slots, cache, page_size, lib=None):
+    """Step a4 into a contiguous [num_pages, page_size, H, D] uint16 cache
+    (modified in place).  Returns the oracle status code."""
+    lib = lib or load()
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    slots = np.ascontiguousarray(slots, dtype=np.int64)
+    assert cache.flags["C_CONTIGUOUS"] and cache.dtype == np.uint16
+    num_pages = cache.shape[0]
+    return lib.oracle_scatter(
+        _p(z, _f64p), z.shape[0], num_heads, D, _p(slots, _i64p),
+        num_pages * page_size, page_size, page_size * num_heads * D,
+        num_heads * D, D, _p(cache, _u16p))
+
+
+def state_update(x, state, lib=None):
+    """Step a5 for one tensor of one sequence; returns the new state rows."""
+    lib = lib or load()
+    x = _u16(x)
+    s = _u16(state).copy()
+    n, C = s.shape
+    lib.oracle_state_update(_p(x, _u16p), C, x.shape[0], _p(s, _u16p), C, C,
+                            n + 1)
+    return s
+
+
+# ---------------------------------------------------------------- whole step
+
+def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
+                   eps, conv_state, slot_mapping, k_cache, v_cache,
+                   state_indices=None, want_z=True, check=True, lib=None):
+    """The whole step (a1..a5) over a varlen batch.
+
+    k, v: uint16 [T, H, D] (or [T, C]); cu_seqlens int32 [S+1];
+    conv_w_*: uint16 [W, C]; gamma_*: float32 [D]; conv_state: uint16
+    [pool, W-1, 2C]; slot_mapping int64 [T]; caches uint16
+    [num_pages, page_size, H, D].  Inputs are not modified: returns
+    dict(k_cache, v_cache, conv_state, z_k, z_v, status) with fresh arrays.
+    """
+    lib = lib or load()
+    k, v = _u16(k), _u16(v)
+    T = k.shape[0]
+    num_pages, page_size, H, D = k_cache.shape
+    C = H * D
+    k2, v2 = k.reshape(T, C), v.reshape(T, C)
+    wk, wv = _u16(conv_w_k), _u16(conv_w_v)
+    W = wk.shape[0]
+    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
+    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    S = cu.shape[0] - 1
+    st = _u16(conv_state).copy()
+    pool = st.shape[0]
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    kc, vc = _u16(k_cache).copy(), _u16(v_cache).copy()
+    si = None if state_indices is None else np.ascontiguousarray(
+        state_indices, dtype=np.int32)
+    zk = np.zeros((T, C), np.float64) if want_z else None
+    zv = np.zeros((T, C), np.float64) if want_z else None
+    rc = lib.oracle_prefill_varlen(
+        _p(k2, _u16p), _p(v2, _u16p), C, T, _p(cu, _i32p), S,
+        _p(wk, _u16p), _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p),
+        float(eps), W, H, D, _p(st if W > 1 else None, _u16p),
+        _p(si, _i32p), pool, _p(sm, _i64p), _p(kc, _u16p), _p(vc, _u16p),
+        num_pages, page_size, page_size * C, C, D, _p(zk, _f64p),
+        _p(zv, _f64p))
+    if check and rc != 0:
+        raise OracleError(rc)
+    return dict(k_cache=kc, v_cache=vc, conv_state=st, z_k=zk, z_v=zv,
+                status=rc)
+
+
+def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
+           slot_mapping, k_cache, v_cache, state_indices=None, want_z=True,
+           check=True, lib=None):
+    """One decode step: one new token per sequence (k, v: [B, H, D])."""
+    B = np.asarray(k).shape[0]
+    cu = np.arange(B + 1, dtype=np.int32)
+    return prefill_varlen(k, v, cu, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
+                          conv_state, slot_mapping, k_cache, v_cache,
+                          state_indices=state_indices, want_z=want_z,
+                          check=check, lib=lib)
+
+
+def decode_direct(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
+                  conv_state, slot_mapping, k_cache, v_cache,
+                  state_indices=None, lib=None):
+    """Decode through the C entry point oracle_decode (same semantics as
+    decode(); kept so both entry points are exercised)."""
+    lib = lib or load()
+    k, v = _u16(k), _u16(v)
+    B = k.shape[0]
+    num_pages, page_size, H, D = k_cache.shape
+    C = H * D
+    k2, v2 = k.reshape(B, C), v.reshape(B, C)
+    wk, wv = _u16(conv_w_k), _u16(conv_w_v)
+    W = wk.shape[0]
+    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
+    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    st = _u16(conv_state).copy()
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    kc, vc = _u16(k_cache).copy(), _u16(v_cache).copy()
+    si = None if state_indices is None else np.ascontiguousarray(
+        state_indices, dtype=np.int32)
+    zk = np.zeros((B, C), np.float64)
+    zv = np.zeros((B, C), np.float64)
+    rc = lib.oracle_decode(
+        _p(k2, _u16p), _p(v2, _u16p), C, B, _p(wk, _u16p), _p(wv, _u16p),
+        _p(gk, _f32p), _p(gv, _f32p), float(eps), W, H, D,
+        _p(st if W > 1 else None, _u16p), _p(si, _i32p), st.shape[0],
+        _p(sm, _i64p), _p(kc, _u16p), _p(vc, _u16p), num_pages, page_size,
+        page_size * C, C, D, _p(zk, _f64p), _p(zv, _f64p))
+    if rc != 0:
+        raise OracleError(rc)
+    return dict(k_cache=kc, v_cache=vc, conv_state=st, z_k=zk, z_v=zv,
+                status=rc)

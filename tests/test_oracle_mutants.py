@@ -1,0 +1,52 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins
+catch every one.  The mistakes are planted on the CPU, in a temporary copy
+of the oracle's C source; the real oracle is never modified."""
+import os
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from tests import pins
+
+# (name, original text, replacement)
+MUTANTS = [
+    ("taps_reversed", "w[(int64_t)j * C + c]", "w[(int64_t)(W - 1 - j) * C + c]"),
+    ("dropped_oldest_tap", "for (int j = 0; j < W; ++j) {", "for (int j = 1; j < W; ++j) {"),
+    ("state_rows_reversed", "s[(W - 1 + q) * state_row_stride + c]", "s[(-1 - q) * state_row_stride + c]"),
+    ("sign_flip", "acc += oracle_bf16_to_double", "acc -= oracle_bf16_to_double"),
+    ("eps_outside_sqrt", "1.0 / sqrt(ss / (double)D + eps)", "1.0 / (sqrt(ss / (double)D) + eps)"),
+    ("sum_not_mean", "1.0 / sqrt(ss / (double)D + eps)", "1.0 / sqrt(ss + eps)"),
+    ("gamma_by_head", "(double)gamma[d]", "(double)gamma[h % D]"),
+    ("state_keeps_oldest", "int64_t q = L - n + j;", "int64_t q = j;"),
+    ("v_uses_k_taps", "(which == 0 ? conv_w_k : conv_w_v)", "(conv_w_k)"),
+    ("v_state_in_k_half", "st + (which == 0 ? 0 : C)", "st + 0"),
+    ("slot_offset_dropped", "int64_t off = slot % page_size;", "int64_t off = 0;"),
+    ("round_truncates", "r = ldexp(rint(ldexp(ax, -q)), q);", "r = ldexp(floor(ldexp(ax, -q)), q);"),
+    ("negative_slot_written", "if (slot < 0) continue;", "if (slot < 0) slot = 0;"),
+    ("head_stride_dropped", "(int64_t)h * stride_head;", "0;"),
+]
+
+
+def _mutant_lib(tmp_path, name, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) >= 1, f"mutant {name}: pattern not found"
+    mutated = src.replace(old, new)
+    path = os.path.join(str(tmp_path), f"mut_{name}.c")
+    with open(path, "w") as f:
+        f.write(mutated)
+    out = os.path.join(str(tmp_path), f"libmut_{name}.so")
+    obuild.build(src=path, out=out)
+    return oracle.load(out)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    lib = _mutant_lib(tmp_path, name, old, new)
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, oracle.OracleError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
