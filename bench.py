@@ -1,0 +1,566 @@
+#!/usr/bin/env python
+"""Benchmark of the fused ShortConv K/V step (tokens/s and achieved HBM GB/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload single|varlen|decode|long|wsweep2|wsweep8]
+
+One step = one pass of the whole step (window assembly + causal conv, RMSNorm,
+bf16 scatter into the paged cache, conv_state update) over one batch,
+through the C ABI.  Default workload: one 8192-token sequence, Hkv=8, D=128,
+W=4, zero state, contiguous cache (page_size 64).
+
+Timing: W warm-up steps, then exactly K steps captured in one CUDA graph and
+replayed once, bracketed by a barrier + synchronize on both sides; an event
+pair around every launch gives the kernel's own duration; max over ranks.
+Inputs rotate over enough buffer sets that each step's bytes exceed L2.
+
+Under torchrun each rank runs its own independent batch (the step shards by
+sequence with no exchange: weak scaling); rank 0 prints one JSON line.
+`--impl reference` times the CPU oracle (test infrastructure) on the same
+workload instead, on rank 0 only.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from short_conv_kv_b200 import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = [os.path.join(ROOT, "short_conv_kv_b200", "csrc", f)
+                  for f in ("common.cuh", "prefill.cuh", "decode.cuh", "sconv_kv.cu")]
+
+
+# ------------------------------------------------------------------ helpers
+
+def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8):
+    """Bytes the step must move: per token K+V rows in and K+V cache rows out
+    plus the slot; per sequence the conv_state rows in and out; per launch
+    the taps and gammas."""
+    C = Hkv * D
+    per_token = 2 * C * 2 + 2 * C * 2 + slot_bytes
+    per_seq = 2 * (W - 1) * 2 * C * 2
+    per_launch = 2 * W * C * 2 + 2 * D * 4
+    return tokens * per_token + seqs * per_seq + per_launch
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0}, "fallback"
+
+
+def profile_traffic(kernel_tag):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel
+    sources are unchanged since the capture (else None)."""
+    path = os.path.join(PROFILE_DIR, f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, throttle reasons) on a thread while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.002):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            # map the CUDA device to its NVML handle by UUID (CUDA and NVML
+            # indices differ under CUDA_VISIBLE_DEVICES)
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ workloads
+
+class Workload:
+    """Device-resident rotating input sets plus host copies for e2e."""
+
+    def __init__(self, name, rank):
+        self.name, self.rank = name, rank
+        seed_shift = 97 * rank
+        if name == "single":
+            self.kind, self.batches = "prefill", [wl.single(seed=2000 + seed_shift)]
+            self.desc = "single-sequence prefill T=8192, Hkv=8, D=128, W=4, zero state, contiguous cache (page 64)"
+        elif name in ("wsweep2", "wsweep4", "wsweep8"):
+            W = int(name[-1])
+            self.kind = "prefill"
+            self.batches = [wl.make_prefill([65536], Hkv=8, D=128, W=W, seed=5100 + W + seed_shift,
+                                            state="zero", page_size=64, permute_pages=True,
+                                            spare_pages=64)]
+            self.desc = f"W-sweep prefill T=65536, W={W}, Hkv=8, D=128, zero state, permuted pages"
+        elif name == "varlen":
+            self.kind, self.batches = "prefill", [wl.varlen(seed=3000 + seed_shift)]
+            self.desc = "varlen prefill 32 seqs U[512,8192], Hkv=8, D=128, W=4, N(0,1) state, permuted pages"
+        elif name == "long":
+            self.kind = "long"
+            self.long = wl.long_context(seed=5000 + seed_shift)
+            self.desc = "long-context chunked prefill 1,048,576 tokens in 65,536-token chunks, W=4, state carried"
+        elif name == "decode":
+            self.kind = "decode"
+            self.dec = wl.decode(seed=4000 + seed_shift)
+            self.desc = "decode 1024 seqs x 1 token, Hkv=8, D=128, W=4, N(0,1) state, 4096-page cache"
+        else:
+            raise SystemExit(f"unknown workload {name}")
+
+    # -- device setup
+    def setup(self, dev):
+        from short_conv_kv_b200 import binding
+        self.binding = binding
+        self.calls_args = []
+        if self.kind == "prefill":
+            b = self.batches[0]
+            self.W, self.Hkv, self.D = b.W, b.Hkv, b.D
+            self.tokens_per_step, self.seqs_per_step = b.num_tokens, b.num_seqs
+            self.bytes_per_step = algorithmic_bytes(b.num_tokens, b.num_seqs, b.W, b.Hkv, b.D)
+            shared = dict(conv_w_k=b.conv_w_k.to(dev), conv_w_v=b.conv_w_v.to(dev),
+                          gamma_k=b.gamma_k.to(dev), gamma_v=b.gamma_v.to(dev))
+            R = max(1, math.ceil(3 * L2_BYTES / self.bytes_per_step))
+            self.rotation = R
+            for r in range(R):
+                self.calls_args.append(dict(
+                    k=b.k.to(dev), v=b.v.to(dev), cu_seqlens=b.cu_seqlens.to(dev),
+                    conv_state=b.conv_state.to(dev), slot_mapping=b.slot_mapping.to(dev),
+                    k_cache=b.empty_cache().to(dev), v_cache=b.empty_cache().to(dev),
+                    eps=b.eps, **shared))
+        elif self.kind == "long":
+            s = self.long
+            self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
+            self.tokens_per_step, self.seqs_per_step = s.chunk, 1
+            self.bytes_per_step = algorithmic_bytes(s.chunk, 1, s.W, s.Hkv, s.D)
+            shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
+                          gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
+                          conv_state=s.initial_state().to(dev),
+                          k_cache=s.empty_cache().to(dev), v_cache=s.empty_cache().to(dev))
+            self.rotation = s.num_chunks
+            for c in range(s.num_chunks):
+                k, v, sm, cu = s.chunk_inputs(c)
+                self.calls_args.append(dict(k=k.to(dev), v=v.to(dev), cu_seqlens=cu.to(dev),
+                                            slot_mapping=sm.to(dev), **shared))
+        else:
+            s = self.dec
+            self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
+            self.tokens_per_step, self.seqs_per_step = s.batch, s.batch
+            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D)
+            shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
+                          gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
+                          k_cache=s.empty_cache().to(dev), v_cache=s.empty_cache().to(dev))
+            R = max(2, math.ceil(3 * L2_BYTES / self.bytes_per_step))
+            self.rotation = R
+            states = [s.conv_state.to(dev) for _ in range(min(R, 16))]
+            for r in range(R):
+                k, v, sm = s.step_inputs(r % 64)
+                self.calls_args.append(dict(k=k.to(dev), v=v.to(dev), slot_mapping=sm.to(dev),
+                                            conv_state=states[r % len(states)], **shared))
+
+    def prepared(self, i, stream):
+        a = self.calls_args[i % len(self.calls_args)]
+        if self.kind == "decode":
+            return self.binding.prepare_decode(
+                a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
+                a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"], a["v_cache"],
+                stream=stream)
+        return self.binding.prepare_prefill_varlen(
+            a["k"], a["v"], a["cu_seqlens"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"],
+            a["gamma_v"], a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"],
+            a["v_cache"], stream=stream)
+
+    def kernel_tag(self):
+        return {"prefill": "prefill_kernel", "long": "prefill_kernel",
+                "decode": "decode_kernel"}[self.kind]
+
+
+# ------------------------------------------------------------------ our arm
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_graph(work, K, Wu, dev, world, local):
+    """Warm-up W eager steps, then K steps captured in one graph (event pair
+    around each launch) and replayed once as the timed region."""
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(Wu):
+            work.prepared(i, stream)()
+    stream.synchronize()
+
+    g = torch.cuda.CUDAGraph()
+    ev_s = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
+    with torch.cuda.graph(g, stream=stream):
+        cap = torch.cuda.current_stream()
+        calls = [work.prepared(i, cap) for i in range(K)]
+        for i in range(K):
+            ev_s[i].record(cap)
+            calls[i]()
+            ev_e[i].record(cap)
+    # one untimed replay uploads the graph and warms it
+    g.replay()
+    torch.cuda.synchronize()
+
+    outer_s = torch.cuda.Event(enable_timing=True)
+    outer_e = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        outer_s.record(stream)
+        with torch.cuda.stream(stream):
+            g.replay()
+        outer_e.record(stream)
+        outer_e.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = outer_s.elapsed_time(outer_e)
+    per_launch = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    del g
+    return total_ms, per_launch, clk.summary()
+
+
+def time_e2e(work, steps, dev):
+    """Same metric end to end through the public API: every step copies its
+    inputs from pinned host memory, runs the step, and reads the written
+    caches and the state back into pinned host memory."""
+    from short_conv_kv_b200 import binding
+    a0 = work.calls_args[0]
+    host_in = {k: a0[k].cpu().pin_memory() for k in ("k", "v", "slot_mapping")}
+    if "cu_seqlens" in a0:
+        host_in["cu_seqlens"] = a0["cu_seqlens"].cpu().pin_memory()
+    host_out = {k: torch.empty(a0[k].shape, dtype=a0[k].dtype, pin_memory=True)
+                for k in ("k_cache", "v_cache", "conv_state")}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        if work.kind == "decode":
+            binding.decode(dev_in["k"], dev_in["v"], a0["conv_w_k"], a0["conv_w_v"],
+                           a0["gamma_k"], a0["gamma_v"], a0["eps"], a0["conv_state"],
+                           dev_in["slot_mapping"], a0["k_cache"], a0["v_cache"], stream=stream)
+        else:
+            binding.prefill_varlen(dev_in["k"], dev_in["v"], dev_in["cu_seqlens"], a0["conv_w_k"],
+                                   a0["conv_w_v"], a0["gamma_k"], a0["gamma_v"], a0["eps"],
+                                   a0["conv_state"], dev_in["slot_mapping"], a0["k_cache"],
+                                   a0["v_cache"], stream=stream)
+        for k in host_out:
+            host_out[k].copy_(a0[k], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+        stream.synchronize()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            step()
+        e.record(stream)
+        e.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return ms, h2d, d2h
+
+
+def _compact(slot_mapping, page_size, Hkv, D):
+    """Dense slots 0..n-1 and a cache just large enough for them: the oracle
+    copies its cache arguments, so timing it against a multi-GB paged cache
+    would time the copy.  Placement is a layout detail; the work per token is
+    the same."""
+    n = int(slot_mapping.shape[0])
+    pages = max(1, -(-n // page_size))
+    cache = np.full((pages, page_size, Hkv, D), wl.SENTINEL_BITS, np.uint16)
+    return np.arange(n, dtype=np.int64), cache
+
+
+def cpu_oracle_baseline(work, budget_s=12.0):
+    """The oracle as it stands (single-threaded C, test infrastructure) on a
+    bounded sample of the same workload: whole batches, repeated until about
+    `budget_s` seconds of CPU work."""
+    import oracle
+    lib = oracle.load()
+    if work.kind == "prefill":
+        b = work.batches[0]
+        sm, cache = _compact(b.slot_mapping, b.page_size, b.Hkv, b.D)
+        args = (wl.bits(b.k), wl.bits(b.v), b.cu_seqlens.numpy(), wl.bits(b.conv_w_k),
+                wl.bits(b.conv_w_v), b.gamma_k.numpy(), b.gamma_v.numpy(), b.eps,
+                wl.bits(b.conv_state), sm, cache, cache.copy())
+        tokens, sample = b.num_tokens, "whole batch"
+        run = lambda: oracle.prefill_varlen(*args, want_z=False, lib=lib)
+    elif work.kind == "long":
+        s = work.long
+        k, v, sm, cu = s.chunk_inputs(0)
+        sm, cache = _compact(sm, s.page_size, s.Hkv, s.D)
+        args = (wl.bits(k), wl.bits(v), cu.numpy(), wl.bits(s.conv_w_k), wl.bits(s.conv_w_v),
+                s.gamma_k.numpy(), s.gamma_v.numpy(), s.eps, wl.bits(s.initial_state()), sm,
+                cache, cache.copy())
+        tokens, sample = k.shape[0], "first 65,536-token chunk"
+        run = lambda: oracle.prefill_varlen(*args, want_z=False, lib=lib)
+    else:
+        s = work.dec
+        k, v, sm = s.step_inputs(0)
+        sm, cache = _compact(sm, s.page_size, s.Hkv, s.D)
+        args = (wl.bits(k), wl.bits(v), wl.bits(s.conv_w_k), wl.bits(s.conv_w_v), s.gamma_k.numpy(),
+                s.gamma_v.numpy(), s.eps, wl.bits(s.conv_state), sm, cache, cache.copy())
+        tokens, sample = s.batch, "decode step 0 (1024 sequences)"
+        run = lambda: oracle.decode(*args, want_z=False, lib=lib)
+    reps, t_tot = 0, 0.0
+    while t_tot < budget_s and reps < 50:
+        t0 = time.perf_counter()
+        run()
+        t_tot += time.perf_counter() - t0
+        reps += 1
+    return {"value": tokens * reps / t_tot, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{sample} x {reps} runs ({t_tot:.1f} s, single thread, dense slots; "
+                      f"host has {os.cpu_count()} cores)"}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    work = Workload(args.workload, rank)
+    work.setup(dev)
+    K, Wu = args.steps, args.warmup
+    total_ms, per_launch, clocks = time_graph(work, K, Wu, dev, world, local)
+    total_ms = max_over_ranks(total_ms, world)
+    kern_ms = statistics.fmean(per_launch)
+    kern_ms = max_over_ranks(kern_ms, world)
+    ms_per_step = total_ms / K
+    value = world * work.tokens_per_step * K / (total_ms / 1e3)
+    e2e_ms, h2d, d2h = time_e2e(work, args.e2e_steps, dev)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    peaks, peak_src = measured_peaks()
+    achieved = work.bytes_per_step / (kern_ms / 1e3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_baseline(work)
+    if rank == 0:
+        line = {
+            "metric": "fused ShortConv-KV tokens/s and achieved HBM GB/s (% of B200 peak)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wu,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": work.desc, "storage": "bf16 in, bf16 cache/state, fp32 math",
+                       "tokens_per_step_per_gpu": work.tokens_per_step,
+                       "seqs_per_step_per_gpu": work.seqs_per_step, "W": work.W,
+                       "num_kv_heads": work.Hkv, "head_dim": work.D,
+                       "parallelism": f"{world} independent replicas (sequence sharding, no collective)",
+                       "l2": f"inputs rotate over {work.rotation} buffer sets "
+                             f"({work.rotation * work.bytes_per_step / 1e6:.0f} MB) > L2",
+                       "timing": "K steps in one CUDA graph replay; event pair per launch"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": profile_traffic(f"{work.kernel_tag()}_{args.workload}"),
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)",
+                         "frac_of_8tbs": achieved / 8000.0,
+                         "algorithmic_bytes_per_launch": work.bytes_per_step,
+                         "kernel_ms_per_launch": kern_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * work.tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """Time the CPU oracle (as it stands) on this arm's workload; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    lib = oracle.load()
+    work = Workload(args.workload, 0)
+    K, Wu = args.steps, args.warmup
+    # per-step sample: the whole batch if K+W steps fit the time budget,
+    # else a prefix of the batch's tokens (same shapes and statistics)
+    if work.kind == "prefill":
+        b = work.batches[0]
+    elif work.kind == "long":
+        s = work.long
+        k, v, sm, cu = s.chunk_inputs(0)
+        b = wl.Batch(W=s.W, Hkv=s.Hkv, D=s.D, eps=s.eps, k=k, v=v, cu_seqlens=cu,
+                     conv_w_k=s.conv_w_k, conv_w_v=s.conv_w_v, gamma_k=s.gamma_k,
+                     gamma_v=s.gamma_v, conv_state=s.initial_state(), slot_mapping=sm,
+                     num_pages=s.num_pages, page_size=s.page_size)
+    else:
+        s = work.dec
+        k, v, sm = s.step_inputs(0)
+        b = wl.Batch(W=s.W, Hkv=s.Hkv, D=s.D, eps=s.eps, k=k, v=v,
+                     cu_seqlens=torch.arange(s.batch + 1, dtype=torch.int32),
+                     conv_w_k=s.conv_w_k, conv_w_v=s.conv_w_v, gamma_k=s.gamma_k,
+                     gamma_v=s.gamma_v, conv_state=s.conv_state, slot_mapping=sm,
+                     num_pages=s.num_pages, page_size=s.page_size)
+    kb, vb = wl.bits(b.k), wl.bits(b.v)
+    cu = b.cu_seqlens.numpy()
+    T = b.num_tokens
+    common = (wl.bits(b.conv_w_k), wl.bits(b.conv_w_v), b.gamma_k.numpy(), b.gamma_v.numpy(), b.eps)
+    state = wl.bits(b.conv_state)
+    dense, cache = _compact(b.slot_mapping, b.page_size, b.Hkv, b.D)
+
+    def one(ntok):
+        # the first sequences' tokens up to ntok (cut inside a sequence if needed)
+        cut = np.minimum(cu, ntok)
+        return oracle.prefill_varlen(kb[:ntok], vb[:ntok], cut.astype(np.int32), *common[:4],
+                                     common[4], state, dense[:ntok], cache, cache,
+                                     want_z=False, lib=lib)
+
+    t0 = time.perf_counter()
+    one(T)
+    full_s = time.perf_counter() - t0
+    budget = 150.0
+    ntok = T if (K + Wu) * full_s <= budget else max(32, int(T * budget / ((K + Wu) * full_s)))
+    for _ in range(Wu):
+        one(ntok)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        one(ntok)
+    dt = time.perf_counter() - t0
+    value = ntok * K / dt
+    line = {
+        "impl": "reference",
+        "metric": "fused ShortConv-KV tokens/s and achieved HBM GB/s (% of B200 peak)",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": Wu,
+        "ms_per_step": dt / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": work.desc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {ntok} of {T} tokens per step, dense slots, single thread; "
+                                   f"host has {os.cpu_count()} cores"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="single",
+                    choices=["single", "varlen", "decode", "long", "wsweep2", "wsweep4", "wsweep8"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * sconv_kv.h -- C ABI of the B200 (sm_100a) fused ShortConv K/V step.
+ *
+ * The step (Inkling architecture; "SGLang and Miles announce day-0 Inkling
+ * support", aib.vote English news item, paragraphs 1-2; "Inkling" model
+ * article on axbrief.com, SConv section):
+ *
+ *   for every token t of sequence i, separately for K and for V:
+ *     y[t,c]   = sum_{j=0}^{W-1} w[j,c] * x[t-W+1+j, c]       causal depthwise
+ *                (rows before the sequence's first token come from the
+ *                 sequence's conv_state, oldest first; w[W-1] meets the
+ *                 current token)
+ *     z[t,h,d] = y[t,h,d] * gamma[d] / sqrt(mean_d y[t,h,:]^2 + eps)
+ *                (RMSNorm over head_dim; the pages only say "normalization",
+ *                 RMSNorm with a learned gamma shared by all heads is the
+ *                 stated reading)
+ *     cache[slot_mapping[t], h, d] = bf16_rne(z[t,h,d])   (skipped if slot < 0)
+ *   and the sequence's conv_state becomes the last W-1 raw input rows of
+ *   (old state ++ the sequence's rows), so the window carries across chunks
+ *   and decode steps (per-request "Mamba/sconv" state pool: Inkling-Small
+ *   SGLang cookbook, section 2 memory-pool paragraph and section 3.5).
+ *
+ * All of it -- conv, norm, cache write, state update -- happens in ONE
+ * kernel pass over HBM.  Arithmetic is fp32 with one rounding to bf16 at the
+ * cache store; state rows are bit copies.
+ *
+ * Conventions for every entry point:
+ *   - tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing, keeps no state between calls and never synchronises;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream); work is enqueued on it and the call returns at once;
+ *   - bf16 tensors are raw 16-bit storage (`void*`); element strides are in
+ *     elements, not bytes;
+ *   - the return value is SCONV_KV_OK or a negative SCONV_KV_ERR_* code; on
+ *     error nothing has been enqueued;
+ *   - problems only visible on the device (a slot beyond the cache, a state
+ *     index beyond the pool, an inconsistent cu_seqlens) never trap: the
+ *     offending token or sequence is skipped and the matching
+ *     SCONV_KV_FLAG_* bit is OR-ed into *err_flag (if err_flag is not NULL);
+ *     the caller clears *err_flag and reads it after synchronising.
+ *
+ * Preconditions the library cannot check without synchronising (results are
+ * unspecified when they are violated): non-negative slots are unique within
+ * a call; state indices are unique within a call; k/v do not alias the
+ * caches or the state; calls that touch the same conv_state or cache rows
+ * are ordered on one stream.
+ */
+#ifndef SCONV_KV_H_
+#define SCONV_KV_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SCONV_KV_API __attribute__((visibility("default")))
+#else
+#define SCONV_KV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+#define SCONV_KV_OK 0
+#define SCONV_KV_ERR_NULL (-1)        /* a required pointer is NULL          */
+#define SCONV_KV_ERR_SHAPE (-2)       /* W, head_dim, heads, counts, strides  */
+#define SCONV_KV_ERR_ALIGN (-3)       /* pointer or stride not 16-byte aligned */
+#define SCONV_KV_ERR_UNSUPPORTED (-4) /* valid but not implemented combination */
+#define SCONV_KV_ERR_CUDA (-5)        /* CUDA reported an error at launch     */
+
+/* ---------------------------------------------------- device-side flag bits */
+#define SCONV_KV_FLAG_SLOT_RANGE 1   /* slot >= num_pages*page_size: skipped  */
+#define SCONV_KV_FLAG_STATE_INDEX 2  /* state index outside the pool: sequence
+                                        skipped (no cache write, no state)   */
+#define SCONV_KV_FLAG_CU_SEQLENS 4   /* cu_seqlens not a partition of
+                                        [0, num_tokens): bad sequences skipped */
+
+/* ------------------------------------------------------------- limits */
+#define SCONV_KV_MAX_W 8             /* conv width W in [1, SCONV_KV_MAX_W]   */
+
+/*
+ * Paged KV cache layout.  Element (slot, h, d) of k_cache (and of v_cache)
+ * lives at
+ *     (slot / page_size) * stride_page + (slot % page_size) * stride_slot
+ *       + h * stride_head + d
+ * elements from the cache base pointer (dim stride 1).  A cache is
+ * num_pages * page_size slots; pages are handed to sequences by the caller
+ * ("prefix pages" of the serving runtime's radix cache, Inkling-Small
+ * cookbook section 3.5), so slot_mapping is an arbitrary scatter.
+ */
+typedef struct sconv_kv_cache_layout_t {
+  int64_t num_pages;
+  int64_t page_size;
+  int64_t num_kv_heads;
+  int64_t head_dim;
+  int64_t stride_page;     /* elements */
+  int64_t stride_slot;     /* elements */
+  int64_t stride_head;     /* elements */
+  int64_t bytes_per_cache; /* bytes spanned by ONE cache (k or v) */
+} sconv_kv_cache_layout_t;
+
+/*
+ * Fill *out with the dense layout [num_pages, page_size, num_kv_heads,
+ * head_dim] (stride_head = head_dim, stride_slot = num_kv_heads*head_dim,
+ * stride_page = page_size*stride_slot).  Callers with another layout (e.g.
+ * K and V interleaved per page) fill the struct themselves.
+ * Host-only; touches no GPU.  Errors: SCONV_KV_ERR_NULL (out == NULL),
+ * SCONV_KV_ERR_SHAPE (a count < 0, page_size < 1, heads < 1, head_dim < 1).
+ */
+SCONV_KV_API int sconv_kv_cache_layout(int64_t num_pages, int64_t page_size,
+                          int num_kv_heads, int head_dim,
+                          sconv_kv_cache_layout_t* out);
+
+/*
+ * Fused ShortConv K/V step over a packed varlen batch (prefill or chunked
+ * prefill; sequences are packed back to back as in flash-attention's varlen
+ * interface).
+ *
+ *  k, v           bf16, token t's row at k + t*row_stride: Hkv*D channels
+ *                 (head-major, then head_dim).  row_stride >= Hkv*D, a
+ *                 multiple of 8 elements; lets k and v be column slices of
+ *                 a fused qkv projection output.  16-byte aligned.
+ *  num_tokens     T, rows of k/v and entries of slot_mapping (>= 0).
+ *  cu_seqlens     int32 [num_seqs+1] on the device: cu[0]=0, non-decreasing,
+ *                 cu[num_seqs]=T.  Sequence i is rows [cu[i], cu[i+1]).
+ *  num_seqs       S >= 0.
+ *  conv_w_k/v     bf16 [W, Hkv*D] taps, row j = tap j (j = W-1 meets the
+ *                 current token).  16-byte aligned.
+ *  gamma_k/v      fp32 [head_dim], shared by all heads.  16-byte aligned.
+ *  eps            RMSNorm epsilon (inside the square root).
+ *  W              conv width, 1..SCONV_KV_MAX_W.
+ *  num_kv_heads   Hkv >= 1.
+ *  head_dim       D in {64, 128, 256}.
+ *  conv_state     bf16 [state_pool_size, W-1, 2*Hkv*D], in/out: raw input
+ *                 rows, oldest first, K channels then V channels.  May be
+ *                 NULL only when W == 1.  16-byte aligned.  New sequences
+ *                 must start from zeroed rows (the caller zeroes them).
+ *  state_indices  int32 [num_seqs] on the device: pool row of sequence i;
+ *                 NULL means sequence i uses pool row i.
+ *  state_pool_size rows in the pool (bounds for state_indices).
+ *  slot_mapping   int64 [T] on the device: cache slot of each token; < 0
+ *                 means "do not write" (padding).
+ *  k_cache, v_cache  bf16 caches described by *layout (host pointer to the
+ *                 struct).  16-byte aligned; stride_head, stride_slot and
+ *                 stride_page multiples of 8 elements.
+ *  err_flag       optional device int; SCONV_KV_FLAG_* bits are OR-ed in.
+ *  stream         cudaStream_t as void*.
+ *
+ * Errors: SCONV_KV_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED, _CUDA as above.
+ * A call with T == 0 or S == 0 enqueues nothing and returns SCONV_KV_OK.
+ */
+SCONV_KV_API int sconv_kv_prefill_varlen(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
+
+/*
+ * Decode specialisation: exactly one new token per sequence (batch
+ * sequences; token b belongs to sequence b, as if cu_seqlens = 0..batch).
+ * Arguments mean what they mean for sconv_kv_prefill_varlen; k and v are
+ * [batch] rows of Hkv*D channels at row_stride.  The sequence's state is
+ * read, the new row is convolved with it, normalised, written to
+ * cache[slot_mapping[b]] and the state is shifted by one row in place.
+ * A call with batch == 0 enqueues nothing.
+ */
+SCONV_KV_API int sconv_kv_decode(
+    const void* k, const void* v, int64_t row_stride, int batch,
+    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+    void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
+
+/* Static text for a status code (never NULL). */
+SCONV_KV_API const char* sconv_kv_strerror(int status);
+
+/* Text of the last CUDA error seen by an entry point on this host thread
+ * ("" if none).  Valid until the next call on the same thread. */
+SCONV_KV_API const char* sconv_kv_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+SCONV_KV_API int sconv_kv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCONV_KV_H_ */

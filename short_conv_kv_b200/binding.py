@@ -1,0 +1,238 @@
+"""ctypes front end of ``libsconvkv.so`` (the fused ShortConv K/V step).
+
+Argument marshalling only: every function takes torch tensors, passes their
+device pointers, sizes and the current CUDA stream to the C ABI declared in
+``include/sconv_kv.h``, and raises on a non-zero status.  All of the step's
+work runs in the library's CUDA kernels; there is no CPU fallback, and if the
+library is missing the import fails loudly.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("SCONV_KV_LIB", _build.LIB)
+
+# status codes and device flag bits (values fixed by include/sconv_kv.h)
+OK = 0
+ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA = -1, -2, -3, -4, -5
+FLAG_SLOT_RANGE, FLAG_STATE_INDEX, FLAG_CU_SEQLENS = 1, 2, 4
+MAX_W = 8
+
+
+class CacheLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "num_pages", "page_size", "num_kv_heads", "head_dim", "stride_page",
+        "stride_slot", "stride_head", "bytes_per_cache")]
+
+
+class SconvKVError(RuntimeError):
+    def __init__(self, code, where):
+        msg = _lib.sconv_kv_strerror(code).decode()
+        if code == ERR_CUDA:
+            msg += ": " + _lib.sconv_kv_last_cuda_error().decode()
+        super().__init__(f"{where} failed with status {code}: {msg}")
+        self.code = code
+
+
+def _load(path):
+    if not os.path.exists(path):
+        raise ImportError(
+            f"CUDA library {path} is not built; run `python -m short_conv_kv_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i64, i32, f32, ip = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                             ctypes.c_float, ctypes.c_void_p)
+    lp = ctypes.POINTER(CacheLayout)
+    lib.sconv_kv_cache_layout.argtypes = [i64, i64, i32, i32, lp]
+    lib.sconv_kv_cache_layout.restype = i32
+    lib.sconv_kv_prefill_varlen.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp,
+        i64, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_prefill_varlen.restype = i32
+    lib.sconv_kv_decode.argtypes = [
+        vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
+        vp, vp, lp, ip, vp]
+    lib.sconv_kv_decode.restype = i32
+    lib.sconv_kv_strerror.argtypes = [i32]
+    lib.sconv_kv_strerror.restype = ctypes.c_char_p
+    lib.sconv_kv_last_cuda_error.argtypes = []
+    lib.sconv_kv_last_cuda_error.restype = ctypes.c_char_p
+    lib.sconv_kv_version.argtypes = []
+    lib.sconv_kv_version.restype = i32
+    return lib
+
+
+_lib = _load(LIB_PATH)
+lib = _lib
+
+
+def strerror(code):
+    return _lib.sconv_kv_strerror(int(code)).decode()
+
+
+def version():
+    return _lib.sconv_kv_version()
+
+
+def cache_layout(num_pages, page_size, num_kv_heads, head_dim):
+    """Dense [num_pages, page_size, Hkv, D] layout (sconv_kv_cache_layout)."""
+    out = CacheLayout()
+    rc = _lib.sconv_kv_cache_layout(int(num_pages), int(page_size),
+                                    int(num_kv_heads), int(head_dim),
+                                    ctypes.byref(out))
+    if rc != OK:
+        raise SconvKVError(rc, "sconv_kv_cache_layout")
+    return out
+
+
+def layout_of(cache):
+    """Layout of a 4-D cache view [num_pages, page_size, Hkv, D] with unit
+    dim stride (e.g. the k or v half of a combined per-page KV buffer)."""
+    if cache.dim() != 4 or cache.stride(3) != 1:
+        raise ValueError("cache must be [num_pages, page_size, Hkv, D] with dim stride 1")
+    P, S, H, D = cache.shape
+    lay = CacheLayout()
+    lay.num_pages, lay.page_size, lay.num_kv_heads, lay.head_dim = P, S, H, D
+    lay.stride_page, lay.stride_slot, lay.stride_head = cache.stride(0), cache.stride(1), cache.stride(2)
+    lay.bytes_per_cache = cache.untyped_storage().nbytes()
+    return lay
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _rows(x, name):
+    """(pointer, row_stride) of a [T, Hkv, D] or [T, Hkv*D] bf16 view whose
+    channels are contiguous."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    if x.dim() == 3:
+        if x.stride(2) != 1 or x.stride(1) != x.shape[2]:
+            raise ValueError(f"{name}: heads and head_dim must be contiguous")
+    elif x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be [T, Hkv, D] or [T, Hkv*D]")
+    C = x[0].numel() if x.shape[0] else x.shape[-1] * (x.shape[1] if x.dim() == 3 else 1)
+    return x.data_ptr(), max(x.stride(0), C)
+
+
+def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
+                   eps, conv_state, slot_mapping, k_cache, v_cache,
+                   state_indices=None, err_flag=None, stream=None,
+                   layout=None):
+    """Fused ShortConv K/V step over a packed varlen batch, on the GPU.
+
+    k, v: bf16 [T, Hkv, D] (rows may be strided slices); cu_seqlens int32
+    [S+1]; conv_w_*: bf16 [W, Hkv*D]; gamma_*: fp32 [D]; conv_state bf16
+    [pool, W-1, 2*Hkv*D] (updated in place); slot_mapping int64 [T];
+    k_cache / v_cache bf16 [num_pages, page_size, Hkv, D] (written in
+    place); state_indices optional int32 [S]; err_flag optional int32 [1].
+    """
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    T = k.shape[0]
+    W = conv_w_k.shape[0]
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    lay = layout if layout is not None else layout_of(k_cache)
+    if v_cache.stride() != k_cache.stride() or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape and strides")
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    rc = _lib.sconv_kv_prefill_varlen(
+        kp, vp, rs, T, _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+        _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
+        float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
+        _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_cache),
+        _ptr(v_cache), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    if rc != OK:
+        raise SconvKVError(rc, "sconv_kv_prefill_varlen")
+
+
+def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
+           slot_mapping, k_cache, v_cache, state_indices=None, err_flag=None,
+           stream=None, layout=None):
+    """Fused ShortConv K/V decode step: one new token per sequence
+    (k, v: bf16 [B, Hkv, D]); same other arguments as prefill_varlen."""
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    B = k.shape[0]
+    W = conv_w_k.shape[0]
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    lay = layout if layout is not None else layout_of(k_cache)
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    rc = _lib.sconv_kv_decode(
+        kp, vp, rs, B, _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+        _ptr(gamma_v), float(eps), W, H, D,
+        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
+        _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
+        _ptr(err_flag), _stream(stream))
+    if rc != OK:
+        raise SconvKVError(rc, "sconv_kv_decode")
+
+
+class PreparedCall:
+    """A pre-marshalled C-ABI call (for tight launch loops and graph
+    capture): the ctypes argument tuple is built once; `__call__` only
+    invokes the C entry point and checks the status."""
+
+    def __init__(self, fn_name, args, keep_alive=()):
+        self._fn = getattr(_lib, fn_name)
+        self._args = tuple(args)
+        self._keep = keep_alive
+        self._name = fn_name
+
+    def __call__(self):
+        rc = self._fn(*self._args)
+        if rc != OK:
+            raise SconvKVError(rc, self._name)
+
+
+def prepare_prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k,
+                           gamma_v, eps, conv_state, slot_mapping, k_cache,
+                           v_cache, state_indices=None, err_flag=None,
+                           stream=None):
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    W = conv_w_k.shape[0]
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    lay = layout_of(k_cache)
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    args = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+            _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
+            ctypes.c_float(eps), W, H, D,
+            _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    return PreparedCall("sconv_kv_prefill_varlen", args, keep_alive=(lay,))
+
+
+def prepare_decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
+                   conv_state, slot_mapping, k_cache, v_cache,
+                   state_indices=None, err_flag=None, stream=None):
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    W = conv_w_k.shape[0]
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    lay = layout_of(k_cache)
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    args = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v),
+            _ptr(gamma_k), _ptr(gamma_v), ctypes.c_float(eps), W, H, D,
+            _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    return PreparedCall("sconv_kv_decode", args, keep_alive=(lay,))
