@@ -74,6 +74,9 @@ extern "C" {
                                         skipped (no cache write, no state)   */
 #define SCONV_KV_FLAG_CU_SEQLENS 4   /* cu_seqlens not a partition of
                                         [0, num_tokens): bad sequences skipped */
+#define SCONV_KV_FLAG_TIMEOUT 8      /* an internal pipeline wait gave up after
+                                        its time limit (about 1 s): the CTA
+                                        stopped early, output incomplete      */
 
 /* ------------------------------------------------------------- limits */
 #define SCONV_KV_MAX_W 8             /* conv width W in [1, SCONV_KV_MAX_W]   */
@@ -147,7 +150,8 @@ SCONV_KV_API int sconv_kv_cache_layout(int64_t num_pages, int64_t page_size,
  *  stream         cudaStream_t as void*.
  *
  * Errors: SCONV_KV_ERR_NULL, _SHAPE, _ALIGN, _UNSUPPORTED, _CUDA as above.
- * A call with T == 0 or S == 0 enqueues nothing and returns SCONV_KV_OK.
+ * A call with T == 0 or S == 0 enqueues nothing and returns SCONV_KV_OK
+ * without examining the pointers (empty tensors may have NULL data).
  */
 SCONV_KV_API int sconv_kv_prefill_varlen(
     const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
@@ -165,7 +169,8 @@ SCONV_KV_API int sconv_kv_prefill_varlen(
  * [batch] rows of Hkv*D channels at row_stride.  The sequence's state is
  * read, the new row is convolved with it, normalised, written to
  * cache[slot_mapping[b]] and the state is shifted by one row in place.
- * A call with batch == 0 enqueues nothing.
+ * A call with batch == 0 enqueues nothing and returns SCONV_KV_OK without
+ * examining the pointers.
  */
 SCONV_KV_API int sconv_kv_decode(
     const void* k, const void* v, int64_t row_stride, int batch,

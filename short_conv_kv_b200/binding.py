@@ -19,7 +19,7 @@ LIB_PATH = os.environ.get("SCONV_KV_LIB", _build.LIB)
 # status codes and device flag bits (values fixed by include/sconv_kv.h)
 OK = 0
 ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA = -1, -2, -3, -4, -5
-FLAG_SLOT_RANGE, FLAG_STATE_INDEX, FLAG_CU_SEQLENS = 1, 2, 4
+FLAG_SLOT_RANGE, FLAG_STATE_INDEX, FLAG_CU_SEQLENS, FLAG_TIMEOUT = 1, 2, 4, 8
 MAX_W = 8
 
 

@@ -44,6 +44,7 @@ struct StepParams {
 constexpr int kFlagSlotRange = 1;
 constexpr int kFlagStateIndex = 2;
 constexpr int kFlagCuSeqlens = 4;
+constexpr int kFlagTimeout = 8;
 
 __device__ __forceinline__ void raise_flag(int* err, int bit) {
   if (err) atomicOr(err, bit);
@@ -98,6 +99,15 @@ __device__ __forceinline__ int64_t slot_row_offset(const StepParams& P,
   if (P.slot_linear) return slot * P.stride_slot;
   const int64_t page = slot / P.page_size;
   return page * P.stride_page + (slot - page * P.page_size) * P.stride_slot;
+}
+
+// Hardware reciprocal square root (PTX rsqrt.approx.ftz.f32, one MUFU op;
+// relative error about 2^-22).  Callers pass x >= eps > 0, so the
+// flush-to-zero and special-value behaviour never matters.
+__device__ __forceinline__ float rsqrt_approx(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Sum of `v` over aligned groups of G lanes (G = D/8 lanes own one head).

@@ -1,0 +1,254 @@
+// Fused ShortConv K/V decode step, streaming version (sm_100a): one new
+// token per sequence.
+//
+// Persistent CTAs (x) over the batch, channel slices of <= 256 groups of 8
+// channels (y).  CTA b handles sequences b, b + ctas, b + 2*ctas, ... (at
+// most kDecMaxSeqs).  In a prologue its threads read every such sequence's
+// state index and slot into shared memory, so the copies need no further
+// index round trips.
+//
+// One ring stage per sequence holds W rows of the CTA's slice: the W-1 old
+// state rows (oldest first) and the new K/V row, brought in by bulk
+// asynchronous copies (thread 0 issues them; completion counted in bytes on
+// the stage's "full" barrier).  Once a stage has landed:
+//   - the new state is exactly stage rows 1..W-1 (old rows 1..W-2, then the
+//     new row), so thread 0 writes it back with bulk shared->global copies
+//     over the rows just read -- the state update never passes through
+//     registers;
+//   - every thread convolves its 8 channels over the W rows, reduces the
+//     head's sum of squares by xor shuffles, and stores its 16 bytes of the
+//     normalised bf16 row into the cache slot.
+// Thread 0 waits until its write-back has finished reading the stage before
+// the stage is released for the next sequence.
+#pragma once
+#include "common.cuh"
+#include "tma.cuh"
+
+namespace sconv {
+
+constexpr int kDecMaxSeqs = 64;  // sequences per CTA (prologue index tables)
+
+struct DecGeom {
+  int slice;      // channel groups per full slice (min(NG, 256))
+  int stages;     // ring depth (sequences in flight per CTA)
+  int ctas;       // CTAs along the batch
+  int smem_ring;  // bytes of the ring
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk store has finished READING shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk store has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// CTAs per SM by register need: four (<= 64 registers) for W <= 4, three
+// for W = 5, two beyond.
+template <int W>
+constexpr int decode_ctas_per_sm() { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
+
+template <int W, int D>
+__global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
+    decode_tma_kernel(const StepParams P, const DecGeom Gm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int G = D / 8;
+  const int B = P.num_seqs;
+  const int NS = Gm.stages;
+
+  const int half = P.NG >> 1;
+  const int g0 = blockIdx.y * Gm.slice;
+  const int cs = min(Gm.slice, P.NG - g0);
+  const int ncw = (cs + 31) >> 5;
+  const int kn = max(0, min(g0 + cs, half) - g0);
+  const int vg0 = max(g0, half);
+  const int vn = max(0, g0 + cs - vg0);
+  const int row_bytes = cs * 16;
+  const int stage_bytes = W * row_bytes;
+  const bool full_slice = (cs == P.NG);
+  const int64_t srow = 2 * static_cast<int64_t>(P.C);
+
+  unsigned char* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Gm.smem_ring);
+  uint64_t* empty = full + NS;
+  long long* s_off = reinterpret_cast<long long*>(empty + NS);  // cache row offset or -1
+  long long* s_si = s_off + kDecMaxSeqs;                        // state row, -1 = skip
+  volatile int* abort = reinterpret_cast<volatile int*>(s_si + kDecMaxSeqs);
+
+  const int lane = threadIdx.x & 31;
+  const int b0 = blockIdx.x;
+  const int nq = b0 < B ? (B - b0 + Gm.ctas - 1) / Gm.ctas : 0;
+  const bool report = blockIdx.y == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncw);
+    }
+    *abort = 0;
+    mbar_init_fence();
+  }
+  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+    const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
+    int64_t si = b;
+    if (W > 1) {
+      si = P.state_indices ? static_cast<int64_t>(P.state_indices[b]) : b;
+      if (si < 0 || si >= P.pool) {
+        if (report) raise_flag(P.err, kFlagStateIndex);
+        si = -1;
+      }
+    }
+    s_si[q] = si;
+    s_off[q] = slot_row_offset(P, P.slots[b], report);
+  }
+  __syncthreads();
+  if (nq == 0) return;
+
+  // ---- producer (thread 0): sequence q -> stage q % NS
+  auto issue = [&](int q) {
+    const int st = q % NS;
+    const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
+    const long long si = s_si[q];
+    if (si < 0) {
+      mbar_arrive(&full[st]);  // skipped sequence: an empty phase
+      return;
+    }
+    mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(stage_bytes));
+    unsigned char* dst = ring + static_cast<size_t>(st) * stage_bytes;
+    if (W > 1) {
+      const uint16_t* sp = P.state + si * (W - 1) * srow;
+      if (full_slice) {
+        bulk_g2s(dst, sp, (W - 1) * row_bytes, &full[st]);
+      } else {
+        for (int r = 0; r < W - 1; ++r) {
+          if (kn) bulk_g2s(dst + r * row_bytes, sp + r * srow + g0 * 8, kn * 16, &full[st]);
+          if (vn)
+            bulk_g2s(dst + r * row_bytes + kn * 16, sp + r * srow + P.C + (vg0 - half) * 8,
+                     vn * 16, &full[st]);
+        }
+      }
+    }
+    unsigned char* xd = dst + (W - 1) * row_bytes;
+    if (kn) bulk_g2s(xd, P.k + b * P.row_stride + g0 * 8, kn * 16, &full[st]);
+    if (vn) bulk_g2s(xd + kn * 16, P.v + b * P.row_stride + (vg0 - half) * 8, vn * 16, &full[st]);
+  };
+  // new state rows 0..W-2 <- stage rows 1..W-1
+  auto write_state = [&](int q) {
+    const long long si = s_si[q];
+    const unsigned char* src = ring + static_cast<size_t>(q % NS) * stage_bytes + row_bytes;
+    uint16_t* sp = P.state + si * (W - 1) * srow;
+    if (full_slice) {
+      bulk_s2g(sp, src, (W - 1) * row_bytes);
+    } else {
+      for (int r = 0; r < W - 1; ++r) {
+        if (kn) bulk_s2g(sp + r * srow + g0 * 8, src + r * row_bytes, kn * 16);
+        if (vn)
+          bulk_s2g(sp + r * srow + P.C + (vg0 - half) * 8, src + r * row_bytes + kn * 16,
+                   vn * 16);
+      }
+    }
+    bulk_commit();
+  };
+  int issued = 0;
+  auto drain = [&]() {  // after giving up: let issued loads land (bounded)
+    for (int d = max(0, issued - NS); d < issued; ++d) {
+      const uint64_t t0 = global_ns();
+      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < Gm.timeout_ns) {
+      }
+    }
+    bulk_wait_all();
+  };
+  if (threadIdx.x == 0)
+    for (; issued < min(NS, nq); ++issued) issue(issued);
+
+  // ---- consumers: this thread's 8 channels
+  const int lg = threadIdx.x;
+  const bool active = lg < cs;
+  const int g = g0 + (active ? lg : 0);
+  const bool isv = g >= half;
+  const int c0 = (isv ? g - half : g) * 8;
+  const int d0 = c0 % D;
+  uint16_t* cache = (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  // taps kept packed (bf16) and widened at use: one token per sequence
+  // makes the extra unpacking cheap, and the saved registers buy occupancy
+  const uint16_t* w = (isv ? P.w_v : P.w_k) + c0;
+  uint4 twp[W];
+#pragma unroll
+  for (int j = 0; j < W; ++j) twp[j] = ld_ro(w + static_cast<int64_t>(j) * P.C);
+  const float* gam = (isv ? P.gamma_v : P.gamma_k) + d0;  // read per sequence (L1)
+
+  for (int q = 0; q < nq; ++q) {
+    const int st = q % NS;
+    if (!mbar_wait(&full[st], (q / NS) & 1, abort, Gm.timeout_ns)) {
+      if (threadIdx.x == 0) {
+        raise_flag(P.err, kFlagTimeout);
+        drain();
+      }
+      return;
+    }
+    const bool run = s_si[q] >= 0;
+    if (run) {
+      if (W > 1 && threadIdx.x == 0) write_state(q);
+      // inactive lanes read column 0 and never store
+      const unsigned char* stage =
+          ring + static_cast<size_t>(st) * stage_bytes + (active ? lg : 0) * 16;
+      float2 acc[4];
+#pragma unroll
+      for (int j = 0; j < W; ++j) {
+        float2 rf[4], tw[4];
+        unpack8(*reinterpret_cast<const uint4*>(stage + j * row_bytes), rf);
+        unpack8(twp[j], tw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = j == 0 ? fmul2(tw[e], rf[e]) : ffma2(tw[e], rf[e], acc[e]);
+      }
+      float2 s2 = fmul2(acc[0], acc[0]);
+      s2 = ffma2(acc[1], acc[1], s2);
+      s2 = ffma2(acc[2], acc[2], s2);
+      s2 = ffma2(acc[3], acc[3], s2);
+      const float ss = group_sum<G>(s2.x + s2.y);
+      const float rn = rsqrt_approx(fmaf(ss, P.inv_d, P.eps));
+      const long long off = s_off[q];
+      if (active && off >= 0) {
+        const float4 ga = __ldg(reinterpret_cast<const float4*>(gam));
+        const float4 gb = __ldg(reinterpret_cast<const float4*>(gam) + 1);
+        const float2 gm[4] = {make_float2(ga.x, ga.y), make_float2(ga.z, ga.w),
+                              make_float2(gb.x, gb.y), make_float2(gb.z, gb.w)};
+        const float2 rr = make_float2(rn, rn);
+        uint4 o;
+        o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
+        o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
+        o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
+        o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
+        st_stream(cache + off, o);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (threadIdx.x == 0 && run && W > 1) bulk_wait_read();  // write-back has read the stage
+      mbar_arrive(&empty[st]);
+    }
+    if (threadIdx.x == 0 && q >= 1 && issued < nq) {
+      if (!mbar_wait(&empty[(q - 1) % NS], ((q - 1) / NS) & 1, abort, Gm.timeout_ns)) {
+        raise_flag(P.err, kFlagTimeout);
+        drain();
+        return;
+      }
+      issue(issued++);
+    }
+  }
+  // the CTA may exit once its write-backs have read shared memory; the
+  // global writes complete with the kernel
+  if (threadIdx.x == 0) bulk_wait_read();
+}
+
+}  // namespace sconv

@@ -1,0 +1,453 @@
+// Fused ShortConv K/V step over a packed varlen batch, streaming version
+// (sm_100a).
+//
+// Work split.  The packed token axis [0, T) is cut into `ctas` contiguous
+// ranges of near-equal length, one per persistent CTA (x), and the channel
+// groups into slices of at most 256 groups of 8 channels (y).  A cut that
+// would fall on positions 1..W-2 of a sequence is moved to position W-1 (or
+// to the sequence's end), so the CTA holding position 0 of a sequence also
+// holds every position whose window reaches into the old conv_state: that
+// CTA is the only reader of the old state and the only writer of the new
+// one, and no inter-CTA synchronisation is needed.
+//
+// Pipeline.  The rows of the CTA's range, preceded by the W-1 rows in front
+// of it when the range starts inside a sequence, stream through a ring of
+// `stages` shared-memory stages of kTmaRows token rows each: one bulk
+// asynchronous copy per row part (K part, V part), completion counted in
+// bytes on the stage's "full" barrier.  Every warp waits on "full", copies
+// the stage's rows into registers and arrives on the stage's "empty"
+// barrier.  Thread 0 is also the producer: it fills the whole ring up front,
+// and in iteration c it refills the stage of chunk c-1 (once every warp has
+// released it) with chunk c-1+stages.  Loads in flight therefore do not
+// occupy registers: each CTA keeps up to a ring's worth of rows requested
+// while it computes.  (No separate producer warp: a 256-thread CTA may use
+// up to 255 registers per thread, which the W <= 8 register window needs.)
+//
+// Consumers.  Consumer thread g owns 8 channels (16 bytes of a row) and walks
+// the rows in token order keeping the last W-1 rows in fp32 registers, as a
+// causal depthwise window.  Per token: conv (packed-fp32 FMAs), per-head sum of
+// squares (in-thread, then xor shuffles over D/8 lanes), rsqrt, gamma, round
+// to bf16, one 16-byte streaming store into the cache slot.  At a sequence
+// start the window is loaded from the sequence's conv_state and the new state
+// (the sequence's last W-1 raw rows) is written by the same thread over the
+// rows it has just read.
+#pragma once
+#include "common.cuh"
+#include "tma.cuh"
+
+namespace sconv {
+
+// Compile-time tuning (defaults chosen by measurement on B200).
+#ifndef SCONV_PREFILL_ROWS
+#define SCONV_PREFILL_ROWS 8
+#endif
+#ifndef SCONV_PREFILL_RING_KB
+#define SCONV_PREFILL_RING_KB 96  // per CTA when two CTAs share an SM
+#endif
+#ifndef SCONV_PREFILL_SMALL_W_PER_SM
+#define SCONV_PREFILL_SMALL_W_PER_SM 2  // CTAs per SM for W <= 4
+#endif
+#ifndef SCONV_PREFILL_EARLY_RELEASE
+#define SCONV_PREFILL_EARLY_RELEASE 0  // copy a stage to registers, then release it
+#endif
+#ifndef SCONV_PREFILL_LAST_WARP_REFILL
+#define SCONV_PREFILL_LAST_WARP_REFILL 0  // the last warp to release a stage refills it
+#endif
+
+constexpr int kTmaMaxGroups = 256;   // channel groups per CTA slice
+constexpr int kTmaRows = SCONV_PREFILL_ROWS;  // token rows per stage
+constexpr int kTmaRingBytes2 = SCONV_PREFILL_RING_KB * 1024;
+constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memory
+
+struct TmaGeom {
+  int slice;      // channel groups per full slice (min(NG, 256))
+  int stages;     // ring depth
+  int ctas;       // persistent CTAs along the token axis
+  int cu_smem;    // cu_seqlens copied to shared memory (num_seqs < kTmaCuSmemMax)
+  int smem_ring;  // bytes of the stage ring
+  unsigned long long timeout_ns;
+};
+
+// Per-token work of one thread: conv of its 8 channels over the window and
+// the new row, then the window shift.  Returns the conv output in acc.
+template <int W>
+__device__ __forceinline__ void conv_step(const float2 (&tw)[W][4], float2 (&win)[W > 1 ? W - 1 : 1][4],
+                                          const uint4& xr, float2 (&acc)[4]) {
+  float2 xf[4];
+  unpack8(xr, xf);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if constexpr (W == 1) {
+      acc[e] = fmul2(tw[0][e], xf[e]);
+    } else {
+      acc[e] = fmul2(tw[0][e], win[0][e]);
+#pragma unroll
+      for (int j = 1; j < W - 1; ++j) acc[e] = ffma2(tw[j][e], win[j][e], acc[e]);
+      acc[e] = ffma2(tw[W - 1][e], xf[e], acc[e]);
+    }
+  }
+  if constexpr (W > 1) {
+#pragma unroll
+    for (int j = 0; j < W - 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) win[j][e] = win[j + 1][e];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) win[W - 2][e] = xf[e];
+  }
+}
+
+// RMSNorm of the head (D/8 lanes), gamma, bf16 rounding, 16-byte store.
+template <int D>
+__device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 (&gm)[4],
+                                           float inv_d, float eps, bool write,
+                                           uint16_t* dst) {
+  float2 s2 = fmul2(acc[0], acc[0]);
+  s2 = ffma2(acc[1], acc[1], s2);
+  s2 = ffma2(acc[2], acc[2], s2);
+  s2 = ffma2(acc[3], acc[3], s2);
+  const float ss = group_sum<D / 8>(s2.x + s2.y);
+  const float rn = rsqrt_approx(fmaf(ss, inv_d, eps));
+  if (write) {
+    const float2 rr = make_float2(rn, rn);
+    uint4 o;
+    o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
+    o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
+    o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
+    o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
+    st_stream(dst, o);
+  }
+}
+
+template <int W, int D, int MINB>
+__global__ void __launch_bounds__(kTmaMaxGroups, MINB)
+    prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int R = kTmaRows;
+  const int S = P.num_seqs;
+  const int T = static_cast<int>(P.num_tokens);
+  const int NS = Gm.stages;
+
+  // ---- channel slice of this CTA
+  const int half = P.NG >> 1;
+  const int g0 = blockIdx.y * Gm.slice;
+  const int cs = min(Gm.slice, P.NG - g0);
+  const int ncw = (cs + 31) >> 5;  // warps (all consume; thread 0 also produces)
+  const int kn = max(0, min(g0 + cs, half) - g0);           // K groups in slice
+  const int vg0 = max(g0, half);
+  const int vn = max(0, g0 + cs - vg0);                     // V groups in slice
+  const int row_bytes = cs * 16;
+
+  unsigned char* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Gm.smem_ring);
+  uint64_t* empty = full + NS;
+  volatile int* abort = reinterpret_cast<volatile int*>(empty + NS);
+  int* s_cu = const_cast<int*>(reinterpret_cast<volatile int*>(empty + NS) + 4);
+#if SCONV_PREFILL_LAST_WARP_REFILL
+  int* rel_cnt = reinterpret_cast<int*>(smem + Gm.smem_ring - 64);  // host reserves 64 B
+#endif
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncw);
+#if SCONV_PREFILL_LAST_WARP_REFILL
+      rel_cnt[s] = 0;
+#endif
+    }
+    *abort = 0;
+    mbar_init_fence();
+  }
+  if (Gm.cu_smem)
+    for (int i = threadIdx.x; i <= S; i += blockDim.x) s_cu[i] = P.cu_seqlens[i];
+  __syncthreads();
+
+  auto cu = [&](int i) -> int { return Gm.cu_smem ? s_cu[i] : __ldg(P.cu_seqlens + i); };
+  // largest i in [0, S-1] with cu[i] <= t
+  auto seq_of = [&](int t) -> int {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu(mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  // start of range b: even cut, moved off positions 1..W-2 of a sequence
+  auto cut = [&](int b) -> int {
+    int s = static_cast<int>((static_cast<int64_t>(b) * T) / Gm.ctas);
+    if (s >= T) return T;
+    if (W > 1) {
+      const int i = seq_of(s);
+      const int a = cu(i), e = cu(i + 1);
+      const int p = s - a;
+      if (p > 0 && p < W - 1) s = a + min(W - 1, e - a);
+      s = min(max(s, 0), T);
+    }
+    return s;
+  };
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    bool ok = cu(0) == 0 && cu(S) == T;
+    for (int i = 0; i < S && ok; ++i) ok = cu(i) <= cu(i + 1);
+    if (!ok) raise_flag(P.err, kFlagCuSeqlens);
+  }
+  const int ta = cut(blockIdx.x);
+  const int tb = max(ta, cut(blockIdx.x + 1));
+  if (ta >= tb) return;
+  const int seq0 = seq_of(ta);
+  // halo rows streamed in front of the range when it starts inside a sequence
+  const int head_rows = (W > 1 && ta > cu(seq0)) ? min(W - 1, ta) : 0;
+  const int first_row = ta - head_rows;
+  const int nrows = tb - first_row;
+  const int nchunks = (nrows + R - 1) / R;
+
+  // =================================================================== producer
+  // Issue chunk c (rows first_row + c*R ...) into stage `st` (= c % NS,
+  // tracked by the caller without a division).
+  auto issue = [&](int c, int st) {
+    const int r0 = first_row + c * R;
+    const int rows = min(R, tb - r0);
+    mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(rows * row_bytes));
+    unsigned char* dst = ring + static_cast<size_t>(st) * R * row_bytes;
+    for (int r = 0; r < rows; ++r) {
+      const int64_t t = r0 + r;
+      if (kn) bulk_g2s(dst, P.k + t * P.row_stride + g0 * 8, kn * 16, &full[st]);
+      if (vn)
+        bulk_g2s(dst + kn * 16, P.v + t * P.row_stride + (vg0 - half) * 8, vn * 16, &full[st]);
+      dst += row_bytes;
+    }
+  };
+  int issued = 0;  // chunks issued so far (thread 0 only)
+  // After giving up, let the copies already issued land before the CTA's
+  // shared memory can be released (bounded as well).
+  auto drain = [&]() {
+    for (int d = max(0, issued - NS); d < issued; ++d) {
+      const uint64_t t0 = global_ns();
+      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < Gm.timeout_ns) {
+      }
+    }
+  };
+  if (threadIdx.x == 0)
+    for (; issued < min(NS, nchunks); ++issued) issue(issued, issued);
+
+  // =================================================================== consumers
+  const int lg = threadIdx.x;  // local channel group
+  const bool active = lg < cs;
+  const int g = g0 + (active ? lg : 0);
+  const bool isv = g >= half;
+  const int c0 = (isv ? g - half : g) * 8;
+  const int d0 = c0 % D;
+  const uint16_t* xbase = (isv ? P.v : P.k) + c0;
+  uint16_t* cache = (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  const int64_t srow = 2 * static_cast<int64_t>(P.C);
+  const int st_chan = (isv ? P.C : 0) + c0;
+
+  float2 tw[W][4];
+  {
+    const uint16_t* w = (isv ? P.w_v : P.w_k) + c0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) unpack8(ld_ro(w + static_cast<int64_t>(j) * P.C), tw[j]);
+  }
+  float2 gm[4];
+  {
+    const float* gam = (isv ? P.gamma_v : P.gamma_k) + d0;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(gam));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(gam) + 1);
+    gm[0] = make_float2(a.x, a.y);
+    gm[1] = make_float2(a.z, a.w);
+    gm[2] = make_float2(b.x, b.y);
+    gm[3] = make_float2(b.z, b.w);
+  }
+  constexpr int NH = W > 1 ? W - 1 : 1;
+  float2 win[NH][4];
+#pragma unroll
+  for (int j = 0; j < NH; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) win[j][e] = make_float2(0.f, 0.f);
+
+  int seq = seq0;
+  int next = (seq + 1 <= S) ? cu(seq + 1) : T;
+  bool skip = false;  // current sequence is not processed (bad state index / cu)
+  const bool report = blockIdx.y == 0 && threadIdx.x == 0;
+  const bool report_slots = blockIdx.y == 0 && warp == 0;  // lane r checks row r's slot
+
+  // Is sequence i processed?  (cu_seqlens entry sane, state index in the
+  // pool.)  A sequence that fails is skipped by every CTA that touches it.
+  auto check_sequence = [&](int i, int64_t& si) -> bool {
+    const int a = cu(i), e = cu(i + 1);
+    if (!(a >= 0 && a <= e && e <= T)) {
+      if (report) raise_flag(P.err, kFlagCuSeqlens);
+      return false;
+    }
+    si = i;
+    if constexpr (W > 1) {
+      si = P.state_indices ? static_cast<int64_t>(P.state_indices[i]) : i;
+      if (si < 0 || si >= P.pool) {
+        if (report) raise_flag(P.err, kFlagStateIndex);
+        return false;
+      }
+    }
+    return true;
+  };
+
+  // Enter sequence `i` at its first token: validate, load the old state into
+  // the window, write the new state.
+  auto start_sequence = [&](int i) {
+    int64_t si;
+    skip = !check_sequence(i, si);
+    if (skip) return;
+    if constexpr (W > 1) {
+      const int a = cu(i), e = cu(i + 1);
+      uint16_t* st = P.state + si * (W - 1) * srow + st_chan;
+      uint4 hb[W - 1];
+#pragma unroll
+      for (int j = 0; j < W - 1; ++j)
+        hb[j] = active ? *reinterpret_cast<const uint4*>(st + j * srow) : make_uint4(0, 0, 0, 0);
+      if (active) {
+        const int L = e - a;
+        const uint16_t* xs = xbase + static_cast<int64_t>(a) * P.row_stride;
+#pragma unroll
+        for (int j = 0; j < W - 1; ++j) {
+          const int q = L - (W - 1) + j;  // row of (old state ++ sequence)
+          uint4 r;
+          if (q >= 0) {
+            r = ld_ro(xs + static_cast<int64_t>(q) * P.row_stride);
+          } else {
+            r = hb[0];
+#pragma unroll
+            for (int m = 1; m < W - 1; ++m)
+              if (m == W - 1 + q) r = hb[m];
+          }
+          *reinterpret_cast<uint4*>(st + j * srow) = r;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < W - 1; ++j) unpack8(hb[j], win[j]);
+    }
+  };
+
+  if (head_rows == 0) {
+    start_sequence(seq);
+  } else {
+    int64_t si;
+    skip = !check_sequence(seq, si);
+  }
+
+  const float eps = P.eps, inv_d = P.inv_d;
+  // inactive lanes read column 0 (and never store): no predicated loads
+  const unsigned char* my_ring = ring + (active ? lg : 0) * 16;
+  // slot_mapping is read one 32-row window ahead of use, lane l holding row
+  // (window start + l), so its load latency hides behind four chunks.
+  constexpr int SW = (32 / R) * R;
+  auto load_slot = [&](int w) -> long long {
+    const int r = first_row + w * SW + lane;
+    return (r >= ta && r < tb) ? P.slots[r] : -1;
+  };
+  long long next_slot = load_slot(0);
+  long long my_off = -1;
+  // stage and phase parity of chunk c (kept without divisions)
+  int s = 0;
+  uint32_t ph = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    if (!mbar_wait(&full[s], ph, abort, Gm.timeout_ns)) {
+      if (threadIdx.x == 0) {
+        raise_flag(P.err, kFlagTimeout);
+        drain();
+      }
+      return;
+    }
+    const int r0 = first_row + c * R;
+    const int rows = min(R, tb - r0);
+    if (c % (SW / R) == 0) {
+      // rows [r0, r0 + 32): lane l holds row r0 + l's cache row offset
+      my_off = slot_row_offset(P, next_slot, report_slots);
+      next_slot = load_slot(c / (SW / R) + 1);
+    }
+    const int sbase = (c % (SW / R)) * R;  // this chunk's first lane
+    const unsigned char* stage = my_ring + static_cast<size_t>(s) * R * row_bytes;
+    bool released = false;
+    if (rows == R && r0 >= ta && next >= r0 + R && !skip) {
+      // fast path: R tokens of one sequence, no halo rows, no branches
+#if SCONV_PREFILL_EARLY_RELEASE
+      uint4 xr[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        xr[r] = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      released = true;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float2 acc[4];
+        conv_step<W>(tw, win, xr[r], acc);
+        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
+        norm_store<D>(acc, gm, inv_d, eps, active && off >= 0, cache + off);
+      }
+#else
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+        float2 acc[4];
+        conv_step<W>(tw, win, xr, acc);
+        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
+        norm_store<D>(acc, gm, inv_d, eps, active && off >= 0, cache + off);
+      }
+#endif
+    } else {
+      for (int r = 0; r < rows; ++r) {
+        const int t = r0 + r;
+        if (t >= next && t >= ta) {
+          // a new sequence starts at t (skip empty ones)
+          while (seq + 1 < S && cu(seq + 1) <= t) ++seq;
+          next = (seq + 1 <= S) ? cu(seq + 1) : T;
+          start_sequence(seq);
+        }
+        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+        float2 acc[4];
+        conv_step<W>(tw, win, xr, acc);
+        if (t < ta) continue;  // halo row: window only
+        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
+        norm_store<D>(acc, gm, inv_d, eps, active && !skip && off >= 0, cache + off);
+      }
+    }
+    __syncwarp();
+#if SCONV_PREFILL_LAST_WARP_REFILL
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&rel_cnt[s], 1) == ncw - 1) {
+        rel_cnt[s] = 0;
+        if (c + NS < nchunks) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue(c + NS, s);
+        }
+      }
+    }
+    (void)released;
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1;
+    }
+    continue;
+#endif
+    if (lane == 0 && !released) mbar_arrive(&empty[s]);  // stage fully consumed
+    if (threadIdx.x == 0 && c >= 1 && issued < nchunks) {
+      // refill the stage of chunk c-1 (issued == c-1+NS lands there) once
+      // every warp has released it
+      const int sp = s == 0 ? NS - 1 : s - 1;
+      const uint32_t pp = s == 0 ? ph ^ 1u : ph;
+      if (!mbar_wait(&empty[sp], pp, abort, Gm.timeout_ns)) {
+        raise_flag(P.err, kFlagTimeout);
+        drain();
+        return;
+      }
+      issue(issued++, sp);
+    }
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1;
+    }
+  }
+}
+
+}  // namespace sconv

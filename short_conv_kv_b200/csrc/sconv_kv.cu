@@ -7,50 +7,66 @@
 
 #include "sconv_kv.h"
 #include "common.cuh"
-#include "decode.cuh"
-#include "prefill.cuh"
+#include "decode_tma.cuh"
+#include "prefill_tma.cuh"
 
 namespace {
 
 using sconv::StepParams;
-using KernelFn = void (*)(StepParams);
 
 thread_local char g_cuda_error[256] = "";
 
-constexpr int kBlock = 256;  // threads per CTA (one 8-channel group each)
-constexpr int kMaxTile = 32;
-constexpr int kMinTile = 8;  // >= SCONV_KV_MAX_W - 1: tile 0 covers the halo
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int W, int D>
-KernelFn prefill_fn() { return sconv::prefill_kernel<W, D>; }
-template <int W, int D>
-KernelFn decode_fn() { return sconv::decode_kernel<W, D>; }
+using TmaFn = void (*)(StepParams, sconv::TmaGeom);
 
-template <int D>
-KernelFn pick_w(bool decode, int W) {
-  switch (W) {
-    case 1: return decode ? decode_fn<1, D>() : prefill_fn<1, D>();
-    case 2: return decode ? decode_fn<2, D>() : prefill_fn<2, D>();
-    case 3: return decode ? decode_fn<3, D>() : prefill_fn<3, D>();
-    case 4: return decode ? decode_fn<4, D>() : prefill_fn<4, D>();
-    case 5: return decode ? decode_fn<5, D>() : prefill_fn<5, D>();
-    case 6: return decode ? decode_fn<6, D>() : prefill_fn<6, D>();
-    case 7: return decode ? decode_fn<7, D>() : prefill_fn<7, D>();
-    case 8: return decode ? decode_fn<8, D>() : prefill_fn<8, D>();
-    default: return nullptr;
-  }
-}
+// W <= 4 fits 128 registers: two CTAs per SM (twice the warps to hide
+// latency); wider windows need more registers and run one CTA per SM.
+template <int W>
+constexpr int prefill_ctas_per_sm() { return W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1; }
 
-KernelFn pick(bool decode, int W, int D) {
-  switch (D) {
-    case 64: return pick_w<64>(decode, W);
-    case 128: return pick_w<128>(decode, W);
-    case 256: return pick_w<256>(decode, W);
-    default: return nullptr;
+template <int W, int D>
+TmaFn prefill_fn() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>()>; }
+using DecFn = void (*)(StepParams, sconv::DecGeom);
+
+template <int W, int D>
+DecFn decode_fn() { return sconv::decode_tma_kernel<W, D>; }
+
+// Kernel instance for (W, D): F<W, D>() over W in 1..8, D in {64, 128, 256}.
+template <typename Fn, template <int, int> class F>
+struct Pick {
+  template <int D>
+  static Fn by_w(int W) {
+    switch (W) {
+      case 1: return F<1, D>::get();
+      case 2: return F<2, D>::get();
+      case 3: return F<3, D>::get();
+      case 4: return F<4, D>::get();
+      case 5: return F<5, D>::get();
+      case 6: return F<6, D>::get();
+      case 7: return F<7, D>::get();
+      case 8: return F<8, D>::get();
+      default: return nullptr;
+    }
   }
-}
+  static Fn get(int W, int D) {
+    switch (D) {
+      case 64: return by_w<64>(W);
+      case 128: return by_w<128>(W);
+      case 256: return by_w<256>(W);
+      default: return nullptr;
+    }
+  }
+};
+template <int W, int D>
+struct DecodeK {
+  static DecFn get() { return decode_fn<W, D>(); }
+};
+template <int W, int D>
+struct PrefillK {
+  static TmaFn get() { return prefill_fn<W, D>(); }
+};
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
@@ -63,6 +79,32 @@ int sm_count() {
     n = 148;
   if (dev < 64) cached[dev] = n;
   return n;
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory (once per kernel and
+// size; host-side attribute, not a stream operation).
+bool smem_attr_set(const void* fn, size_t bytes) {
+  static const void* done_fn[256];
+  static size_t done_bytes[256];
+  static int n_done = 0;
+  for (int i = 0; i < n_done; ++i)
+    if (done_fn[i] == fn && done_bytes[i] >= bytes) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  for (int i = 0; i < n_done; ++i)
+    if (done_fn[i] == fn) {
+      done_bytes[i] = bytes;
+      return true;
+    }
+  if (n_done < 256) {
+    done_fn[n_done] = fn;
+    done_bytes[n_done] = bytes;
+    ++n_done;
+  }
+  return true;
 }
 
 // Checks shared by both entry points; fills the common part of P.
@@ -121,10 +163,9 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
   return SCONV_KV_OK;
 }
 
-int launch(KernelFn fn, dim3 grid, dim3 block, StepParams* P, void* stream) {
-  void* args[] = {P};
-  cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), grid, block, args, 0,
-                                   static_cast<cudaStream_t>(stream));
+int launch(const void* fn, dim3 grid, dim3 block, void** args, size_t smem, void* stream) {
+  cudaError_t e =
+      cudaLaunchKernel(fn, grid, block, args, smem, static_cast<cudaStream_t>(stream));
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
@@ -135,11 +176,6 @@ int launch(KernelFn fn, dim3 grid, dim3 block, StepParams* P, void* stream) {
   return SCONV_KV_OK;
 }
 
-// Threads per CTA: all channel groups when they fit, in whole warps.
-dim3 block_for(int NG) {
-  const int t = NG >= kBlock ? kBlock : ((NG + 31) / 32) * 32;
-  return dim3(t);
-}
 
 }  // namespace
 
@@ -185,15 +221,17 @@ int sconv_kv_prefill_varlen(
     const int32_t* state_indices, int64_t state_pool_size,
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
     const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  // an empty call enqueues nothing; its pointers are not examined (empty
+  // tensors may have NULL data pointers)
+  if (num_seqs < 0 || num_tokens < 0 || num_tokens > INT32_MAX) return SCONV_KV_ERR_SHAPE;
+  if (num_seqs == 0 || num_tokens == 0) return SCONV_KV_OK;
   StepParams P;
   int rc = validate_common(k, v, row_stride, conv_w_k, conv_w_v, gamma_k, gamma_v, W,
                            num_kv_heads, head_dim, conv_state, state_pool_size,
                            slot_mapping, k_cache, v_cache, layout, &P);
   if (rc != SCONV_KV_OK) return rc;
   if (!cu_seqlens) return SCONV_KV_ERR_NULL;
-  if (num_seqs < 0 || num_tokens < 0 || num_tokens > INT32_MAX) return SCONV_KV_ERR_SHAPE;
-  if (num_seqs == 0 || num_tokens == 0) return SCONV_KV_OK;
-  KernelFn fn = pick(false, W, head_dim);
+  TmaFn fn = Pick<TmaFn, PrefillK>::get(W, head_dim);
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
 
   P.num_tokens = num_tokens;
@@ -203,21 +241,40 @@ int sconv_kv_prefill_varlen(
   P.state_indices = state_indices;
   P.err = err_flag;
 
-  // Tile length: spread the tokens over one wave of resident CTAs when
-  // there are few, cap the tile when there are many (more, shorter CTAs
-  // balance better at the tail).  Tile >= W-1 keeps the old state inside
-  // the first tile of each sequence.
-  const dim3 block = block_for(P.NG);
-  const int64_t ctas_y = (P.NG + block.x - 1) / block.x;
-  const int64_t resident = static_cast<int64_t>(sm_count()) * (W <= 4 ? 2 : 1);
-  int64_t tile = (num_tokens * ctas_y + resident - 1) / resident;
-  if (tile > kMaxTile) tile = kMaxTile;
-  if (tile < kMinTile) tile = kMinTile;
-  P.tile = static_cast<int>(tile);
-  const int64_t grid_x = num_tokens / tile + num_seqs;
-  if (grid_x > INT32_MAX || ctas_y > 65535) return SCONV_KV_ERR_SHAPE;
-  return launch(fn, dim3(static_cast<unsigned>(grid_x), static_cast<unsigned>(ctas_y)), block,
-                &P, stream);
+  // Geometry: channel slices of <= 256 groups (y), one thread per group
+  // (thread 0 also issues the copies); two CTAs per SM with a ~96 KB ring
+  // each (W <= 4) or one with ~192 KB; as many persistent CTAs per slice as
+  // are resident (x), each streaming a contiguous token range of at least
+  // one stage.
+  sconv::TmaGeom G;
+  G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
+  const int ctas_y = (P.NG + G.slice - 1) / G.slice;
+  const int stage_bytes = sconv::kTmaRows * G.slice * 16;
+  const int per_sm = W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1;  // = prefill_ctas_per_sm<W>()
+  int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
+  G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
+  G.smem_ring = G.stages * stage_bytes;
+#if SCONV_PREFILL_LAST_WARP_REFILL
+  G.smem_ring += 64;  // release counters (placed just below the barriers)
+#endif
+  G.cu_smem = num_seqs < sconv::kTmaCuSmemMax ? 1 : 0;
+  G.timeout_ns = 1000000000ull;
+  const int64_t resident = static_cast<int64_t>(sm_count()) * per_sm;
+  int64_t ctas = resident / ctas_y;
+  const int64_t by_tokens = (num_tokens + sconv::kTmaRows - 1) / sconv::kTmaRows;
+  if (ctas > by_tokens) ctas = by_tokens;
+  if (ctas < 1) ctas = 1;
+  G.ctas = static_cast<int>(ctas);
+  const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 16 +
+                      (G.cu_smem ? 4 * static_cast<size_t>(num_seqs + 1) : 0);
+  if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
+    return SCONV_KV_ERR_CUDA;
+  }
+  const dim3 block(((G.slice + 31) / 32) * 32);
+  void* args[] = {&P, &G};
+  return launch(reinterpret_cast<const void*>(fn), dim3(G.ctas, ctas_y), block, args, smem,
+                stream);
 }
 
 int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
@@ -227,25 +284,51 @@ int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
                     int64_t state_pool_size, const int64_t* slot_mapping, void* k_cache,
                     void* v_cache, const sconv_kv_cache_layout_t* layout, int* err_flag,
                     void* stream) {
+  if (batch < 0) return SCONV_KV_ERR_SHAPE;
+  if (batch == 0) return SCONV_KV_OK;  // nothing enqueued, pointers not examined
   StepParams P;
   int rc = validate_common(k, v, row_stride, conv_w_k, conv_w_v, gamma_k, gamma_v, W,
                            num_kv_heads, head_dim, conv_state, state_pool_size,
                            slot_mapping, k_cache, v_cache, layout, &P);
   if (rc != SCONV_KV_OK) return rc;
-  if (batch < 0) return SCONV_KV_ERR_SHAPE;
-  if (batch == 0) return SCONV_KV_OK;
-  KernelFn fn = pick(true, W, head_dim);
+  DecFn fn = Pick<DecFn, DecodeK>::get(W, head_dim);
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
   P.num_tokens = batch;
   P.num_seqs = batch;
   P.eps = eps;
   P.state_indices = state_indices;
   P.err = err_flag;
-  const dim3 block = block_for(P.NG);
-  const int64_t ctas_y = (P.NG + block.x - 1) / block.x;
+
+  // Geometry: channel slices of <= 256 groups (y), one thread per group;
+  // four CTAs per SM (fewer for W > 4) sharing ~192 KB of ring
+  // (one stage = one sequence's W rows); enough CTAs (x) that each handles
+  // at most kDecMaxSeqs sequences, and at least one resident wave.
+  sconv::DecGeom G;
+  G.slice = P.NG < 256 ? P.NG : 256;
+  const int ctas_y = (P.NG + G.slice - 1) / G.slice;
+  const int stage_bytes = W * G.slice * 16;
+  const int per_sm = W <= 4 ? 4 : (W == 5 ? 3 : 2);  // = decode_ctas_per_sm<W>()
+  int stages = (192 * 1024 / per_sm) / stage_bytes;
+  G.stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  G.smem_ring = G.stages * stage_bytes;
+  G.timeout_ns = 1000000000ull;
+  int64_t ctas = static_cast<int64_t>(sm_count()) * per_sm / ctas_y;
+  const int64_t need = (static_cast<int64_t>(batch) + sconv::kDecMaxSeqs - 1) / sconv::kDecMaxSeqs;
+  if (ctas < need) ctas = need;
+  if (ctas > batch) ctas = batch;
+  if (ctas < 1) ctas = 1;
+  G.ctas = static_cast<int>(ctas);
   if (ctas_y > 65535) return SCONV_KV_ERR_SHAPE;
-  return launch(fn, dim3(static_cast<unsigned>(batch), static_cast<unsigned>(ctas_y)), block,
-                &P, stream);
+  const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages +
+                      2 * sconv::kDecMaxSeqs * sizeof(long long) + 16;
+  if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
+    return SCONV_KV_ERR_CUDA;
+  }
+  const dim3 block(((G.slice + 31) / 32) * 32);
+  void* args[] = {&P, &G};
+  return launch(reinterpret_cast<const void*>(fn), dim3(G.ctas, ctas_y), block, args, smem,
+                stream);
 }
 
 }  // extern "C"

@@ -86,9 +86,10 @@ def test_validation_codes_on_host():
     lay = b.cache_layout(16, 16, 2, 64)
     lay.stride_slot = 132
     assert _call_prefill(b, layout=ctypes.byref(lay)) == b.ERR_ALIGN
-    # empty calls enqueue nothing and succeed
+    # empty calls enqueue nothing and succeed, whatever the pointers
     assert _call_prefill(b, num_tokens=0) == b.OK
     assert _call_prefill(b, num_seqs=0) == b.OK
+    assert _call_prefill(b, num_tokens=0, k=None, v=None, slots=None, cu=None) == b.OK
 
 
 def test_decode_validation_on_host():
@@ -109,7 +110,7 @@ def test_decode_validation_on_host():
     bad[12] = None  # W = 4 needs a state
     assert b.lib.sconv_kv_decode(*bad) == b.ERR_NULL
     bad = list(base)
-    bad[9], bad[12] = 1, None  # W = 1: no state needed; batch 0 -> no-op
+    bad[0], bad[1], bad[15] = None, None, None  # batch 0: pointers not examined
     assert b.lib.sconv_kv_decode(*bad[:3], 0, *bad[4:]) == b.OK
 
 
