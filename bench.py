@@ -246,8 +246,8 @@ class Workload:
             a["v_cache"], stream=stream)
 
     def kernel_tag(self):
-        return {"prefill": "prefill_kernel", "long": "prefill_kernel",
-                "decode": "decode_kernel"}[self.kind]
+        return {"prefill": "prefill_tma_kernel", "long": "prefill_tma_kernel",
+                "decode": "decode_tma_kernel"}[self.kind]
 
 
 # ------------------------------------------------------------------ our arm
@@ -273,9 +273,11 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Slowest rank's value (NCCL needs a device tensor, gloo a host one)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    on_gpu = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
