@@ -79,6 +79,17 @@ __device__ __forceinline__ void st_stream(uint16_t* p, const uint4& v) {
   __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
+// The same store under a predicate, as one predicated instruction (no
+// branch around it).
+__device__ __forceinline__ void st_stream_if(bool pred, uint16_t* p, const uint4& v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %0, 0;\n\t"
+      "@q st.global.cs.v4.u32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"(static_cast<int>(pred)),
+      "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+      : "memory");
+}
+
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return __ffma2_rn(a, b, c);
 }

@@ -10,8 +10,8 @@
 // CTA is the only reader of the old state and the only writer of the new
 // one, and no inter-CTA synchronisation is needed.
 //
-// Pipeline.  The rows of the CTA's range, preceded by the W-1 rows in front
-// of it when the range starts inside a sequence, stream through a ring of
+// Pipeline.  The rows of the CTA's range (the W-1 rows in front of a range
+// that starts inside a sequence are read directly) stream through a ring of
 // `stages` shared-memory stages of kTmaRows token rows each: one bulk
 // asynchronous copy per row part (K part, V part), completion counted in
 // bytes on the stage's "full" barrier.  Every warp waits on "full", copies
@@ -56,8 +56,19 @@ namespace sconv {
 
 constexpr int kTmaMaxGroups = 256;   // channel groups per CTA slice
 constexpr int kTmaRows = SCONV_PREFILL_ROWS;  // token rows per stage
+
+// Measured on B200: with W <= 4 (two CTAs per SM, 128 registers) the fast
+// path is unrolled by 4 and gamma is read from shared memory per token,
+// which frees the registers the unrolled tokens need; wider windows run one
+// CTA per SM with room for an 8-token unroll and gamma in registers.
+template <int W>
+__host__ __device__ constexpr bool gamma_in_smem() { return W <= 4; }
+template <int W>
+__host__ __device__ constexpr int fast_unroll() { return W <= 4 ? 4 : 8; }
 constexpr int kTmaRingBytes2 = SCONV_PREFILL_RING_KB * 1024;
 constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memory
+constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 8;  // per-warp slot offsets
+constexpr int kTmaGammaBytes = kTmaMaxGroups * 32;  // 8 gammas per thread (W <= 4)
 
 struct TmaGeom {
   int slice;      // channel groups per full slice (min(NG, 256))
@@ -96,6 +107,22 @@ __device__ __forceinline__ void conv_step(const float2 (&tw)[W][4], float2 (&win
   }
 }
 
+// 8 gammas from shared memory, read at the point of use (kept out of
+// registers: the loads are volatile, so they are not hoisted).
+__device__ __forceinline__ void lds_gamma(const float* g, float2 (&gm)[4]) {
+  float4 a, b;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w)
+               : "r"(smem_u32(g)));
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(b.x), "=f"(b.y), "=f"(b.z), "=f"(b.w)
+               : "r"(smem_u32(g + 4)));
+  gm[0] = make_float2(a.x, a.y);
+  gm[1] = make_float2(a.z, a.w);
+  gm[2] = make_float2(b.x, b.y);
+  gm[3] = make_float2(b.z, b.w);
+}
+
 // RMSNorm of the head (D/8 lanes), gamma, bf16 rounding, 16-byte store.
 template <int D>
 __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 (&gm)[4],
@@ -107,15 +134,13 @@ __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 
   s2 = ffma2(acc[3], acc[3], s2);
   const float ss = group_sum<D / 8>(s2.x + s2.y);
   const float rn = rsqrt_approx(fmaf(ss, inv_d, eps));
-  if (write) {
-    const float2 rr = make_float2(rn, rn);
-    uint4 o;
-    o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
-    o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
-    o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
-    o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
-    st_stream(dst, o);
-  }
+  const float2 rr = make_float2(rn, rn);
+  uint4 o;
+  o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
+  o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
+  o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
+  o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
+  st_stream_if(write, dst, o);
 }
 
 template <int W, int D, int MINB>
@@ -143,8 +168,12 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   volatile int* abort = reinterpret_cast<volatile int*>(empty + NS);
   int* s_cu = const_cast<int*>(reinterpret_cast<volatile int*>(empty + NS) + 4);
 #if SCONV_PREFILL_LAST_WARP_REFILL
-  int* rel_cnt = reinterpret_cast<int*>(smem + Gm.smem_ring - 64);  // host reserves 64 B
+  int* rel_cnt = reinterpret_cast<int*>(smem + Gm.smem_ring - kTmaOffTableBytes - 64);
 #endif
+  // per-warp table of the cache row offsets of the current 32-row window
+  // (host reserves 8 warps x 32 x 8 bytes right below the barriers)
+  long long* warp_off =
+      reinterpret_cast<long long*>(smem + Gm.smem_ring - kTmaOffTableBytes) + (threadIdx.x >> 5) * 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -196,9 +225,11 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   const int tb = max(ta, cut(blockIdx.x + 1));
   if (ta >= tb) return;
   const int seq0 = seq_of(ta);
-  // halo rows streamed in front of the range when it starts inside a sequence
-  const int head_rows = (W > 1 && ta > cu(seq0)) ? min(W - 1, ta) : 0;
-  const int first_row = ta - head_rows;
+  // a range that starts inside a sequence needs the W-1 rows in front of it
+  // (its halo); they are read directly below, so the ring holds exactly the
+  // range's own rows and every full chunk can take the fast path
+  const bool mid_sequence = (W > 1 && ta > cu(seq0));
+  const int first_row = ta;
   const int nrows = tb - first_row;
   const int nchunks = (nrows + R - 1) / R;
 
@@ -249,15 +280,24 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
 #pragma unroll
     for (int j = 0; j < W; ++j) unpack8(ld_ro(w + static_cast<int64_t>(j) * P.C), tw[j]);
   }
+  // gamma: this thread's 8 values, either staged in its own 32 bytes of
+  // shared memory (read per token) or held in registers
+  float* my_gamma = reinterpret_cast<float*>(smem + Gm.smem_ring - kTmaOffTableBytes -
+                                             kTmaGammaBytes) + threadIdx.x * 8;
   float2 gm[4];
   {
     const float* gam = (isv ? P.gamma_v : P.gamma_k) + d0;
     const float4 a = __ldg(reinterpret_cast<const float4*>(gam));
     const float4 b = __ldg(reinterpret_cast<const float4*>(gam) + 1);
-    gm[0] = make_float2(a.x, a.y);
-    gm[1] = make_float2(a.z, a.w);
-    gm[2] = make_float2(b.x, b.y);
-    gm[3] = make_float2(b.z, b.w);
+    if constexpr (gamma_in_smem<W>()) {
+      reinterpret_cast<float4*>(my_gamma)[0] = a;
+      reinterpret_cast<float4*>(my_gamma)[1] = b;
+    } else {
+      gm[0] = make_float2(a.x, a.y);
+      gm[1] = make_float2(a.z, a.w);
+      gm[2] = make_float2(b.x, b.y);
+      gm[3] = make_float2(b.z, b.w);
+    }
   }
   constexpr int NH = W > 1 ? W - 1 : 1;
   float2 win[NH][4];
@@ -327,14 +367,34 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
   };
 
-  if (head_rows == 0) {
+  if (!mid_sequence) {
     start_sequence(seq);
   } else {
     int64_t si;
     skip = !check_sequence(seq, si);
+    if constexpr (W > 1) {
+      // halo: rows ta-(W-1) .. ta-1 of the same sequence (the cut rule puts
+      // ta at position >= W-1, so they are never state rows)
+#pragma unroll
+      for (int j = 0; j < W - 1; ++j) {
+        const int64_t q = static_cast<int64_t>(ta) - (W - 1) + j;
+        const uint4 h = (active && q >= 0) ? ld_ro(xbase + q * P.row_stride) : make_uint4(0, 0, 0, 0);
+        unpack8(h, win[j]);
+      }
+    }
   }
 
   const float eps = P.eps, inv_d = P.inv_d;
+#define NORM_STORE(pred)                                              \
+  do {                                                                \
+    if constexpr (gamma_in_smem<W>()) {                               \
+      float2 gs[4];                                                   \
+      lds_gamma(my_gamma, gs);                                        \
+      norm_store<D>(acc, gs, inv_d, eps, (pred), cache + off);        \
+    } else {                                                          \
+      norm_store<D>(acc, gm, inv_d, eps, (pred), cache + off);        \
+    }                                                                 \
+  } while (0)
   // inactive lanes read column 0 (and never store): no predicated loads
   const unsigned char* my_ring = ring + (active ? lg : 0) * 16;
   // slot_mapping is read one 32-row window ahead of use, lane l holding row
@@ -342,10 +402,9 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   constexpr int SW = (32 / R) * R;
   auto load_slot = [&](int w) -> long long {
     const int r = first_row + w * SW + lane;
-    return (r >= ta && r < tb) ? P.slots[r] : -1;
+    return r < tb ? P.slots[r] : -1;
   };
   long long next_slot = load_slot(0);
-  long long my_off = -1;
   // stage and phase parity of chunk c (kept without divisions)
   int s = 0;
   uint32_t ph = 0;
@@ -360,15 +419,18 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     const int r0 = first_row + c * R;
     const int rows = min(R, tb - r0);
     if (c % (SW / R) == 0) {
-      // rows [r0, r0 + 32): lane l holds row r0 + l's cache row offset
-      my_off = slot_row_offset(P, next_slot, report_slots);
+      // rows [r0, r0 + SW): lane l writes row r0 + l's cache row offset
+      __syncwarp();
+      warp_off[lane] = slot_row_offset(P, next_slot, report_slots);
+      __syncwarp();
       next_slot = load_slot(c / (SW / R) + 1);
     }
     const int sbase = (c % (SW / R)) * R;  // this chunk's first lane
     const unsigned char* stage = my_ring + static_cast<size_t>(s) * R * row_bytes;
     bool released = false;
-    if (rows == R && r0 >= ta && next >= r0 + R && !skip) {
-      // fast path: R tokens of one sequence, no halo rows, no branches
+    if (next >= r0 + rows && !skip) {
+      // fast path: up to R tokens of one sequence, no branches (rows past
+      // the end of the range compute on stale data and are not stored)
 #if SCONV_PREFILL_EARLY_RELEASE
       uint4 xr[R];
 #pragma unroll
@@ -381,23 +443,23 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       for (int r = 0; r < R; ++r) {
         float2 acc[4];
         conv_step<W>(tw, win, xr[r], acc);
-        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
-        norm_store<D>(acc, gm, inv_d, eps, active && off >= 0, cache + off);
+        const long long off = warp_off[sbase + r];
+        NORM_STORE(active && r < rows && off >= 0);
       }
 #else
-#pragma unroll
+#pragma unroll fast_unroll<W>()
       for (int r = 0; r < R; ++r) {
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
         float2 acc[4];
         conv_step<W>(tw, win, xr, acc);
-        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
-        norm_store<D>(acc, gm, inv_d, eps, active && off >= 0, cache + off);
+        const long long off = warp_off[sbase + r];
+        NORM_STORE(active && r < rows && off >= 0);
       }
 #endif
     } else {
       for (int r = 0; r < rows; ++r) {
         const int t = r0 + r;
-        if (t >= next && t >= ta) {
+        if (t >= next) {
           // a new sequence starts at t (skip empty ones)
           while (seq + 1 < S && cu(seq + 1) <= t) ++seq;
           next = (seq + 1 <= S) ? cu(seq + 1) : T;
@@ -406,9 +468,8 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
         float2 acc[4];
         conv_step<W>(tw, win, xr, acc);
-        if (t < ta) continue;  // halo row: window only
-        const long long off = __shfl_sync(kFullMask, my_off, sbase + r);
-        norm_store<D>(acc, gm, inv_d, eps, active && !skip && off >= 0, cache + off);
+        const long long off = warp_off[sbase + r];
+        NORM_STORE(active && !skip && off >= 0);
       }
     }
     __syncwarp();
@@ -448,6 +509,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       ph ^= 1;
     }
   }
+#undef NORM_STORE
 }
 
 }  // namespace sconv

@@ -253,9 +253,10 @@ int sconv_kv_prefill_varlen(
   const int per_sm = W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1;  // = prefill_ctas_per_sm<W>()
   int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
-  G.smem_ring = G.stages * stage_bytes;
+  // + per-warp slot-offset tables + per-thread gammas
+  G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes + sconv::kTmaGammaBytes;
 #if SCONV_PREFILL_LAST_WARP_REFILL
-  G.smem_ring += 64;  // release counters (placed just below the barriers)
+  G.smem_ring += 64;  // release counters
 #endif
   G.cu_smem = num_seqs < sconv::kTmaCuSmemMax ? 1 : 0;
   G.timeout_ns = 1000000000ull;
