@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     *abort = 0;
     mbar_init_fence();
   }
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
   for (int q = threadIdx.x; q < nq; q += blockDim.x) {
     const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
     int64_t si = b;
@@ -111,14 +112,12 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     s_si[q] = si;
     s_off[q] = slot_row_offset(P, P.slots[b], report);
   }
-  __syncthreads();
   if (nq == 0) return;
 
-  // ---- producer (thread 0): sequence q -> stage q % NS
-  auto issue = [&](int q) {
+  // ---- producer (thread 0): sequence q (pool row si, -1 = skip) -> stage q % NS
+  auto issue = [&](int q, long long si) {
     const int st = q % NS;
     const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
-    const long long si = s_si[q];
     if (si < 0) {
       mbar_arrive(&full[st]);  // skipped sequence: an empty phase
       return;
@@ -168,8 +167,19 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     }
     bulk_wait_all();
   };
-  if (threadIdx.x == 0)
-    for (; issued < min(NS, nq); ++issued) issue(issued);
+  // With identity state indices thread 0 knows every pool row at once and
+  // starts the copies before the index tables are even complete; otherwise
+  // it waits for the tables.
+  const bool identity = (W == 1) || P.state_indices == nullptr;
+  if (identity && threadIdx.x == 0)
+    for (; issued < min(NS, nq); ++issued) {
+      const int64_t b = b0 + static_cast<int64_t>(issued) * Gm.ctas;
+      issue(issued, (W == 1 || b < P.pool) ? b : -1);
+    }
+  __syncthreads();
+  if (!identity && threadIdx.x == 0)
+    for (; issued < min(NS, nq); ++issued) issue(issued, s_si[issued]);
+  if (threadIdx.x == 0 && issued == nq) allow_dependent_launch();
 
   // ---- consumers: this thread's 8 channels
   const int lg = threadIdx.x;
@@ -243,7 +253,8 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
         drain();
         return;
       }
-      issue(issued++);
+      issue(issued, s_si[issued]);
+      if (++issued == nq) allow_dependent_launch();
     }
   }
   // the CTA may exit once its write-backs have read shared memory; the

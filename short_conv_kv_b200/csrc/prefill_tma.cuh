@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     *abort = 0;
     mbar_init_fence();
   }
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
   if (Gm.cu_smem)
     for (int i = threadIdx.x; i <= S; i += blockDim.x) s_cu[i] = P.cu_seqlens[i];
   __syncthreads();
@@ -259,8 +260,10 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       }
     }
   };
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0) {
     for (; issued < min(NS, nchunks); ++issued) issue(issued, issued);
+    if (issued == nchunks) allow_dependent_launch();
+  }
 
   // =================================================================== consumers
   const int lg = threadIdx.x;  // local channel group
@@ -503,6 +506,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
         return;
       }
       issue(issued++, sp);
+      if (issued == nchunks) allow_dependent_launch();
     }
     if (++s == NS) {
       s = 0;

@@ -163,9 +163,21 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
   return SCONV_KV_OK;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start
+// while the previous kernel in the stream drains; it waits for that kernel
+// (griddepcontrol.wait) before touching global memory.
 int launch(const void* fn, dim3 grid, dim3 block, void** args, size_t smem, void* stream) {
-  cudaError_t e =
-      cudaLaunchKernel(fn, grid, block, args, smem, static_cast<cudaStream_t>(stream));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),

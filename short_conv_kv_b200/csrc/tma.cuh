@@ -69,6 +69,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their memory is visible (a no-op when the launch has
+// no programmatic dependency).  Must precede every global-memory access.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the next grid in the stream start launching (its CTAs still wait in
+// grid_dependency_wait() until this grid has completed).
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // One bulk copy global -> this CTA's shared memory, completion signalled on
 // `bar` as transaction bytes.  dst, src 16-byte aligned; bytes % 16 == 0.
 // (Plain load: no cluster multicast.)
