@@ -81,6 +81,20 @@ def load(path=None):
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     lib.oracle_round_bf16_array.argtypes = [_f64p, _i64, _u16p]
     lib.oracle_round_bf16_array.restype = None
+    _u8p = ctypes.POINTER(ctypes.c_uint8)
+    lib.oracle_double_to_e4m3.argtypes = [ctypes.c_double]
+    lib.oracle_double_to_e4m3.restype = ctypes.c_uint8
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_e4m3_array.argtypes = [_f64p, _i64, _u8p]
+    lib.oracle_e4m3_array.restype = None
+    lib.oracle_mx_block.argtypes = [_f32p, _int, _u8p, _u8p]
+    lib.oracle_mx_block.restype = None
+    lib.oracle_prefill_varlen_mxfp8.argtypes = (
+        [_u16p, _u16p, _i64, _i64, _i32p, _int, _u16p, _u16p, _f32p, _f32p,
+         ctypes.c_double, _int, _int, _int, _u16p, _i32p, _i64, _i64p,
+         _u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64, _i64, _f64p, _f64p])
+    lib.oracle_prefill_varlen_mxfp8.restype = _int
     if path == _build.LIB:
         _lib = lib
     return lib
@@ -264,3 +278,76 @@ def decode_direct(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
         raise OracleError(rc)
     return dict(k_cache=kc, v_cache=vc, conv_state=st, z_k=zk, z_v=zv,
                 status=rc)
+
+
+# ---------------------------------------------------------------- MXFP8 store
+
+def e4m3_from_f64(x, lib=None):
+    """FP8 E4M3 codes (nearest even, saturating at +-448) of float64 values."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, np.uint8)
+    lib.oracle_e4m3_array(_p(x, _f64p), x.size,
+                          out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
+
+
+def e4m3_to_f64(codes, lib=None):
+    lib = lib or load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_to_double(int(t)) for t in c.reshape(-1)],
+                    dtype=np.float64).reshape(c.shape)
+
+
+def mx_block(values_f32, lib=None):
+    """Quantise one block of float32 values -> (codes uint8[n], scale uint8)."""
+    lib = lib or load()
+    v = np.ascontiguousarray(values_f32, dtype=np.float32)
+    codes = np.zeros(v.shape[0], np.uint8)
+    scale = np.zeros(1, np.uint8)
+    _u8p = ctypes.POINTER(ctypes.c_uint8)
+    lib.oracle_mx_block(_p(v, _f32p), v.shape[0], codes.ctypes.data_as(_u8p),
+                        scale.ctypes.data_as(_u8p))
+    return codes, int(scale[0])
+
+
+def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
+                         eps, conv_state, slot_mapping, num_pages, page_size,
+                         state_indices=None, check=True, lib=None):
+    """The step with the MXFP8 store into dense caches: data uint8
+    [num_pages, page_size, H, D], scales uint8 [num_pages, page_size, H, D/32]
+    (fresh, zero-filled).  Returns dict(k_data, k_scale, v_data, v_scale,
+    conv_state, z_k, z_v, status)."""
+    lib = lib or load()
+    k, v = _u16(k), _u16(v)
+    T = k.shape[0]
+    wk, wv = _u16(conv_w_k), _u16(conv_w_v)
+    W, C = wk.shape
+    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
+    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    D = gk.shape[0]
+    H = C // D
+    k2, v2 = k.reshape(T, C), v.reshape(T, C)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    S = cu.shape[0] - 1
+    st = _u16(conv_state).copy()
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    si = None if state_indices is None else np.ascontiguousarray(state_indices, dtype=np.int32)
+    kd = np.zeros((num_pages, page_size, H, D), np.uint8)
+    vd = np.zeros_like(kd)
+    ks = np.zeros((num_pages, page_size, H, D // 32), np.uint8)
+    vs = np.zeros_like(ks)
+    zk = np.zeros((T, C), np.float64)
+    zv = np.zeros((T, C), np.float64)
+    _u8p = ctypes.POINTER(ctypes.c_uint8)
+    rc = lib.oracle_prefill_varlen_mxfp8(
+        _p(k2, _u16p), _p(v2, _u16p), C, T, _p(cu, _i32p), S, _p(wk, _u16p),
+        _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p), float(eps), W, H, D,
+        _p(st if W > 1 else None, _u16p), _p(si, _i32p), st.shape[0],
+        _p(sm, _i64p), kd.ctypes.data_as(_u8p), ks.ctypes.data_as(_u8p),
+        vd.ctypes.data_as(_u8p), vs.ctypes.data_as(_u8p), num_pages, page_size,
+        page_size * C, C, D, _p(zk, _f64p), _p(zv, _f64p))
+    if check and rc != 0:
+        raise OracleError(rc)
+    return dict(k_data=kd, k_scale=ks, v_data=vd, v_scale=vs, conv_state=st,
+                z_k=zk, z_v=zv, status=rc)

@@ -350,3 +350,140 @@ int oracle_decode(const uint16_t* k, const uint16_t* v, int64_t row_stride,
 void oracle_round_bf16_array(const double* x, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_bf16(x[i]);
 }
+
+/* ==================================================================== */
+/* MXFP8 (block-scaled) cache store.                                    */
+/*                                                                      */
+/* Source: "Inkling-Small" SGLang cookbook, section 3.6 (Long Context):  */
+/* KV entries can be stored as block-scaled MXFP8 instead of BF16,      */
+/* about doubling the tokens a pool holds.  The pages give no block     */
+/* size or scale format; MXFP8 is read as the OCP Microscaling format:  */
+/* blocks of 32 consecutive elements (here: 32 channels of one head)    */
+/* share one power-of-two scale X = 2^s stored as an E8M0 byte (s+127), */
+/* and each element is stored as FP8 E4M3 of v/X.  The shared exponent  */
+/* is s = floor(log2(max|v|)) - 8 (8 = exponent of E4M3's largest       */
+/* normal, 448 = 1.75 * 2^8), clamped to [-127, 127]; elements are      */
+/* rounded to nearest even and saturated to +-448.  The quantisation    */
+/* decisions are taken on the normalised value rounded to binary32 (the */
+/* kernel's precision), so both sides decide from the same kind of      */
+/* number.                                                              */
+/* ==================================================================== */
+
+/* FP8 E4M3 (sign, 4-bit exponent with bias 7, 3-bit mantissa; largest
+ * finite 448, no infinities, subnormals M * 2^-9) of a double: nearest
+ * even on the E4M3 grid, magnitudes at or above 448 saturate to 448. */
+uint8_t oracle_double_to_e4m3(double x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs(x);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);            /* a = m * 2^e, m in [0.5, 1): floor(log2 a) = e-1 */
+  int q = (e - 1) - 3;     /* grid spacing 2^q for normals */
+  if (q < -9) q = -9;      /* subnormal spacing 2^-9 */
+  double r = ldexp(rint(ldexp(a, -q)), q);
+  if (r > 448.0) r = 448.0;
+  if (r == 0.0) return sign;
+  frexp(r, &e);
+  int E = (e - 1) + 7;
+  if (E <= 0) return (uint8_t)(sign | (uint8_t)ldexp(r, 9)); /* M * 2^-9 */
+  int M = (int)(ldexp(r, -(e - 1)) * 8.0) - 8;
+  return (uint8_t)(sign | (uint8_t)(E << 3) | (uint8_t)M);
+}
+
+double oracle_e4m3_to_double(uint8_t c) {
+  const double sign = (c & 0x80) ? -1.0 : 1.0;
+  const int E = (c >> 3) & 0xF, M = c & 0x7;
+  if (E == 0xF && M == 0x7) return NAN;
+  if (E == 0) return sign * ldexp((double)M, -9);
+  return sign * ldexp(1.0 + M / 8.0, E - 7);
+}
+
+/* Quantise one block of n binary32 values: shared exponent -> *scale
+ * (E8M0 code), element codes -> codes[0..n). */
+void oracle_mx_block(const float* v, int n, uint8_t* codes, uint8_t* scale) {
+  double amax = 0.0;
+  for (int i = 0; i < n; ++i)
+    if (fabs((double)v[i]) > amax) amax = fabs((double)v[i]);
+  int s;
+  if (amax < ldexp(1.0, -126)) {
+    s = -127; /* zero or subnormal block: the smallest scale */
+  } else {
+    int e;
+    frexp(amax, &e);
+    s = (e - 1) - 8;
+    if (s < -127) s = -127;
+    if (s > 127) s = 127;
+  }
+  *scale = (uint8_t)(s + 127);
+  for (int i = 0; i < n; ++i) codes[i] = oracle_double_to_e4m3(ldexp((double)v[i], -s));
+}
+
+/* The whole step with the MXFP8 store (steps a1-a3 and a5 as in
+ * oracle_prefill_varlen; a4 writes E4M3 codes and E8M0 block scales).
+ * Data caches: uint8, element (slot, h, d) at the usual element offset;
+ * scale caches: uint8, block (slot, h, b) at (page*stride_page +
+ * off*stride_slot + h*stride_head)/32 + b (all strides multiples of 32).
+ * z_k / z_v (optional) receive the unrounded double values. */
+int oracle_prefill_varlen_mxfp8(
+    const uint16_t* k, const uint16_t* v, int64_t row_stride,
+    int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
+    const uint16_t* conv_w_k, const uint16_t* conv_w_v, const float* gamma_k,
+    const float* gamma_v, double eps, int W, int num_heads, int D,
+    uint16_t* conv_state, const int32_t* state_indices,
+    int64_t state_pool_size, const int64_t* slot_mapping, uint8_t* k_data,
+    uint8_t* k_scale, uint8_t* v_data, uint8_t* v_scale, int64_t num_pages,
+    int64_t page_size, int64_t stride_page, int64_t stride_slot,
+    int64_t stride_head, double* z_k, double* z_v) {
+  if (D % 32 || stride_page % 32 || stride_slot % 32 || stride_head % 32)
+    return ORACLE_ERR_ARG;
+  const int C = num_heads * D;
+  /* run the bf16 oracle for z and the state (its bf16 caches are scratch) */
+  const int64_t num_slots = num_pages * page_size;
+  uint16_t* scratch_k = (uint16_t*)calloc((size_t)(num_slots > 0 ? num_slots : 1) * (size_t)C, 2);
+  uint16_t* scratch_v = (uint16_t*)calloc((size_t)(num_slots > 0 ? num_slots : 1) * (size_t)C, 2);
+  double* zk = z_k ? z_k : (double*)malloc(sizeof(double) * (size_t)(num_tokens ? num_tokens : 1) * (size_t)C);
+  double* zv = z_v ? z_v : (double*)malloc(sizeof(double) * (size_t)(num_tokens ? num_tokens : 1) * (size_t)C);
+  if (!scratch_k || !scratch_v || !zk || !zv) {
+    free(scratch_k); free(scratch_v);
+    if (!z_k) free(zk);
+    if (!z_v) free(zv);
+    return ORACLE_ERR_NOMEM;
+  }
+  int rc = oracle_prefill_varlen(
+      k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+      gamma_k, gamma_v, eps, W, num_heads, D, conv_state, state_indices,
+      state_pool_size, slot_mapping, scratch_k, scratch_v, num_slots, 1,
+      C, C, D, zk, zv);
+  free(scratch_k);
+  free(scratch_v);
+  if (rc == ORACLE_OK) {
+    float block[32];
+    for (int64_t t = 0; t < num_tokens; ++t) {
+      const int64_t slot = slot_mapping[t];
+      if (slot < 0 || slot >= num_slots) continue;
+      const int64_t page = slot / page_size, off = slot % page_size;
+      for (int which = 0; which < 2; ++which) {
+        const double* z = (which == 0 ? zk : zv) + t * C;
+        uint8_t* data = which == 0 ? k_data : v_data;
+        uint8_t* scl = which == 0 ? k_scale : v_scale;
+        for (int h = 0; h < num_heads; ++h) {
+          const int64_t base = page * stride_page + off * stride_slot + h * stride_head;
+          for (int b = 0; b < D / 32; ++b) {
+            for (int i = 0; i < 32; ++i) block[i] = (float)z[h * D + b * 32 + i];
+            oracle_mx_block(block, 32, data + base + b * 32, scl + base / 32 + b);
+          }
+        }
+      }
+    }
+  }
+  if (!z_k) free(zk);
+  if (!z_v) free(zv);
+  return rc;
+}
+
+/* Vector helper for the Python side: E4M3 codes of n doubles. */
+void oracle_e4m3_array(const double* x, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_e4m3(x[i]);
+}

@@ -347,3 +347,121 @@ ALL_PINS = [
     pin_untouched_slots, pin_state_update, pin_scale_invariance,
     pin_page_permutation, pin_errors, pin_decode_entry,
 ]
+
+
+# ------------------------------------------------------------ MXFP8 store pins
+
+def _e4m3_table():
+    """All finite E4M3 values by code, built from the format's definition
+    (sign, exponent bias 7, 3 mantissa bits, E=15/M=7 is NaN)."""
+    vals = {}
+    for c in range(256):
+        E, M = (c >> 3) & 0xF, c & 7
+        if E == 0xF and M == 7:
+            continue
+        mag = (M / 8.0) * 2.0 ** -6 if E == 0 else (1 + M / 8.0) * 2.0 ** (E - 7)
+        vals[c] = -mag if c & 0x80 else mag
+    return vals
+
+
+def pin_e4m3_rounding(lib):
+    """E4M3 rounding: nearest value of the code table with ties to the even
+    code (brute force), torch's float8_e4m3fn conversion for in-range
+    float32 inputs, saturation to +-448, subnormal ties, round trips."""
+    table = _e4m3_table()
+    pos = sorted((v, c) for c, v in table.items() if v > 0 or c == 0)
+    rng = np.random.default_rng(3)
+    xs = np.concatenate([rng.standard_normal(3000) * 30, rng.standard_normal(1000) * 1e-2,
+                         np.array([v for v, _ in pos]),
+                         np.array([(a[0] + b[0]) / 2 for a, b in zip(pos[:-1], pos[1:])])])
+    got = oracle.e4m3_from_f64(xs, lib=lib)
+    for x, g in zip(xs, got):
+        a = abs(x)
+        if a >= 448:
+            exp = 0x7E
+        else:
+            best = min(pos, key=lambda vc: (abs(vc[0] - a), vc[1] & 1))
+            exp = best[1]
+        if x < 0 or (x == 0 and np.signbit(x)):
+            exp |= 0x80
+        assert int(g) == exp, (x, int(g), exp)
+    x32 = (rng.standard_normal(4000) * 50).astype(np.float32)
+    x32 = x32[np.abs(x32) < 448]
+    ref = torch.from_numpy(x32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_from_f64(x32.astype(np.float64), lib=lib), ref)
+    assert int(oracle.e4m3_from_f64(np.array([1e9]), lib=lib)[0]) == 0x7E
+    assert int(oracle.e4m3_from_f64(np.array([-500.0]), lib=lib)[0]) == 0xFE
+    assert int(oracle.e4m3_from_f64(np.array([2.0 ** -10]), lib=lib)[0]) == 0x00  # tie -> even 0
+    assert int(oracle.e4m3_from_f64(np.array([3 * 2.0 ** -10]), lib=lib)[0]) == 0x02  # tie -> even 2
+    codes = np.array([c for c in table if c != 0x80], np.uint8)
+    back = oracle.e4m3_from_f64(oracle.e4m3_to_f64(codes, lib=lib), lib=lib)
+    assert np.array_equal(back, codes)
+
+
+def pin_mx_block(lib):
+    """Block scaling: the scale is 2^(floor(log2 amax) - 8) (checked against
+    math.frexp), a power-of-two amax maps to 256 (code 0x78), a zero block
+    takes the smallest scale, scaling the block by 2^j shifts the scale
+    code by j and keeps the element codes, and every element is the E4M3
+    rounding of v / 2^s."""
+    import math
+    rng = np.random.default_rng(4)
+    for _ in range(200):
+        v = (rng.standard_normal(32) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32)
+        codes, scale = oracle.mx_block(v, lib=lib)
+        amax = float(np.max(np.abs(v.astype(np.float64))))
+        m, e = math.frexp(amax)
+        s = max(-127, min(127, (e - 1) - 8))
+        assert scale == s + 127, (amax, scale, s)
+        assert np.array_equal(codes, oracle.e4m3_from_f64(v.astype(np.float64) * 2.0 ** -s, lib=lib))
+        for j in (-3, 2, 7):
+            c2, s2 = oracle.mx_block((v.astype(np.float64) * 2.0 ** j).astype(np.float32), lib=lib)
+            assert s2 == scale + j and np.array_equal(c2, codes)
+    v = np.zeros(32, np.float32)
+    v[5] = 2.0 ** 3
+    v[6] = -2.0 ** 1
+    codes, scale = oracle.mx_block(v, lib=lib)
+    assert scale == (3 - 8) + 127 and codes[5] == 0x78 and codes[6] == (0x80 | 0x68)
+    codes, scale = oracle.mx_block(np.zeros(32, np.float32), lib=lib)
+    assert scale == 0 and not codes.any()
+    # the largest element lands in [256, 448]: values in (448, 512) saturate
+    v = np.full(32, 1.9, np.float32)
+    codes, scale = oracle.mx_block(v, lib=lib)
+    assert scale == (0 - 8) + 127 and np.all(codes == 0x7E)
+
+
+def pin_mxfp8_step(lib):
+    """The MXFP8 store writes, for every written slot, head and 32-channel
+    block, exactly the block quantisation of the step's normalised values
+    rounded to binary32, leaves unnamed slots zero, and updates the state
+    like the bf16 step."""
+    b = wl.make_prefill([20, 9], Hkv=2, D=64, W=4, seed=61, state="normal",
+                        page_size=8, spare_pages=2)
+    sm = b.slot_mapping.numpy().copy()
+    sm[3] = -1
+    out = oracle.prefill_varlen_mxfp8(
+        _bits(b.k), _bits(b.v), b.cu_seqlens.numpy(), _bits(b.conv_w_k), _bits(b.conv_w_v),
+        b.gamma_k.numpy(), b.gamma_v.numpy(), b.eps, _bits(b.conv_state), sm,
+        b.num_pages, b.page_size, lib=lib)
+    ref = _run(lib, b, slots=sm)
+    assert np.array_equal(out["conv_state"], ref["conv_state"])
+    assert np.array_equal(out["z_k"], ref["z_k"]) and np.array_equal(out["z_v"], ref["z_v"])
+    H, D = b.Hkv, b.D
+    for which in ("k", "v"):
+        data = out[f"{which}_data"].reshape(-1, H, D)
+        scl = out[f"{which}_scale"].reshape(-1, H, D // 32)
+        z = out[f"z_{which}"].reshape(-1, H, D)
+        written = np.zeros(data.shape[0], bool)
+        for t, slot in enumerate(sm):
+            if slot < 0:
+                continue
+            written[slot] = True
+            for h in range(H):
+                for blk in range(D // 32):
+                    c, s = oracle.mx_block(z[t, h, blk * 32:(blk + 1) * 32].astype(np.float32), lib=lib)
+                    assert np.array_equal(data[slot, h, blk * 32:(blk + 1) * 32], c)
+                    assert scl[slot, h, blk] == s
+        assert not data[~written].any() and not scl[~written].any()
+
+
+ALL_PINS += [pin_e4m3_rounding, pin_mx_block, pin_mxfp8_step]

@@ -25,6 +25,11 @@ MUTANTS = [
     ("round_truncates", "r = ldexp(rint(ldexp(ax, -q)), q);", "r = ldexp(floor(ldexp(ax, -q)), q);"),
     ("negative_slot_written", "if (slot < 0) continue;", "if (slot < 0) slot = 0;"),
     ("head_stride_dropped", "(int64_t)h * stride_head;", "0;"),
+    ("mx_emax_7", "s = (e - 1) - 8;", "s = (e - 1) - 7;"),
+    ("mx_ceil_log2", "s = (e - 1) - 8;", "s = e - 8;"),
+    ("e4m3_overflow_nan", "if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 448.0) return (uint8_t)(sign | 0x7F);"),
+    ("e4m3_truncates", "double r = ldexp(rint(ldexp(a, -q)), q);", "double r = ldexp(floor(ldexp(a, -q)), q);"),
+    ("e4m3_subnormal_grid", "if (q < -9) q = -9;", "if (q < -10) q = -10;"),
 ]
 
 
