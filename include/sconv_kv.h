@@ -180,6 +180,51 @@ SCONV_KV_API int sconv_kv_decode(
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
     const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
 
+/*
+ * MXFP8 cache store ("Inkling-Small" SGLang cookbook, section 3.6 Long
+ * Context: KV entries stored as block-scaled MXFP8 instead of BF16, about
+ * twice the tokens per pool).  The page gives no block size or scale
+ * format; this follows the OCP Microscaling (MX) format:
+ *   - each head's D channels form D/32 blocks of 32 consecutive channels;
+ *   - a block stores one E8M0 scale byte s + 127, X = 2^s with
+ *     s = floor(log2(max |z| over the block)) - 8 (8 = exponent of E4M3's
+ *     largest normal, 448 = 1.75 * 2^8), s = -127 for an all-zero or
+ *     subnormal block;
+ *   - each element stores the FP8 E4M3 code of z / X, rounded to nearest
+ *     even, magnitudes beyond 448 saturated to 448;
+ *   - z is the normalised value of the bf16 entry points, in binary32; the
+ *     rounding decisions are taken on it.
+ *
+ * Arguments are those of sconv_kv_prefill_varlen / sconv_kv_decode, except
+ * the caches:
+ *   k_data, v_data    uint8 E4M3 codes; element (slot, h, d) at the element
+ *                     offset given by *layout (1 byte per element).
+ *                     16-byte aligned.
+ *   k_scale, v_scale  uint8 E8M0 scales; block (slot, h, b) at
+ *                     (page*stride_page + off*stride_slot + h*stride_head)/32
+ *                     + b.  The layout's strides must be multiples of 32.
+ * Errors and flags as for the bf16 entry points (SCONV_KV_ERR_ALIGN also
+ * when a stride is not a multiple of 32).
+ */
+SCONV_KV_API int sconv_kv_prefill_varlen_mxfp8(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout, int* err_flag,
+    void* stream);
+
+SCONV_KV_API int sconv_kv_decode_mxfp8(
+    const void* k, const void* v, int64_t row_stride, int batch,
+    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+    void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout, int* err_flag,
+    void* stream);
+
 /* Static text for a status code (never NULL). */
 SCONV_KV_API const char* sconv_kv_strerror(int status);
 

@@ -57,6 +57,14 @@ def _load(path):
         vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
         vp, vp, lp, ip, vp]
     lib.sconv_kv_decode.restype = i32
+    lib.sconv_kv_prefill_varlen_mxfp8.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp,
+        i64, vp, vp, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_prefill_varlen_mxfp8.restype = i32
+    lib.sconv_kv_decode_mxfp8.argtypes = [
+        vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
+        vp, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_decode_mxfp8.restype = i32
     lib.sconv_kv_strerror.argtypes = [i32]
     lib.sconv_kv_strerror.restype = ctypes.c_char_p
     lib.sconv_kv_last_cuda_error.argtypes = []
@@ -185,6 +193,70 @@ def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
         raise SconvKVError(rc, "sconv_kv_decode")
 
 
+def _mx_layout(k_data, k_scale, v_data, v_scale):
+    """Layout of MXFP8 caches: data uint8 [num_pages, page_size, Hkv, D]
+    (unit dim stride), scales uint8 [num_pages, page_size, Hkv, D/32] whose
+    strides are the data strides / 32."""
+    for t, n in ((k_data, "k_data"), (v_data, "v_data"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t.dtype != torch.uint8:
+            raise TypeError(f"{n} must be uint8")
+    lay = layout_of(k_data)
+    if v_data.stride() != k_data.stride() or v_data.shape != k_data.shape:
+        raise ValueError("k_data and v_data must have the same shape and strides")
+    P, S, H, D = k_data.shape
+    want = (P, S, H, D // 32)
+    for sc in (k_scale, v_scale):
+        if tuple(sc.shape) != want or sc.stride(3) != 1 or any(
+                sc.stride(i) * 32 != k_data.stride(i) for i in range(3)):
+            raise ValueError("scale caches must be [num_pages, page_size, Hkv, D/32] with "
+                             "strides equal to the data strides / 32")
+    return lay
+
+
+def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
+                         eps, conv_state, slot_mapping, k_data, k_scale, v_data, v_scale,
+                         state_indices=None, err_flag=None, stream=None):
+    """The fused step with the block-scaled MXFP8 cache store (E4M3 codes in
+    k_data/v_data, one E8M0 scale byte per 32 channels in k_scale/v_scale)."""
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    lay = _mx_layout(k_data, k_scale, v_data, v_scale)
+    W = conv_w_k.shape[0]
+    H, D = k_data.shape[2], k_data.shape[3]
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    rc = _lib.sconv_kv_prefill_varlen_mxfp8(
+        kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+        _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v), float(eps), W, H, D,
+        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(slot_mapping),
+        _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale), ctypes.byref(lay),
+        _ptr(err_flag), _stream(stream))
+    if rc != OK:
+        raise SconvKVError(rc, "sconv_kv_prefill_varlen_mxfp8")
+
+
+def decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
+                 slot_mapping, k_data, k_scale, v_data, v_scale, state_indices=None,
+                 err_flag=None, stream=None):
+    """Decode step with the MXFP8 cache store (one new token per sequence)."""
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    lay = _mx_layout(k_data, k_scale, v_data, v_scale)
+    W = conv_w_k.shape[0]
+    H, D = k_data.shape[2], k_data.shape[3]
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    rc = _lib.sconv_kv_decode_mxfp8(
+        kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+        _ptr(gamma_v), float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
+        _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
+        _ptr(v_data), _ptr(v_scale), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    if rc != OK:
+        raise SconvKVError(rc, "sconv_kv_decode_mxfp8")
+
+
 class PreparedCall:
     """A pre-marshalled C-ABI call (for tight launch loops and graph
     capture): the ctypes argument tuple is built once; `__call__` only
@@ -236,3 +308,37 @@ def prepare_decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
             _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
             ctypes.byref(lay), _ptr(err_flag), _stream(stream))
     return PreparedCall("sconv_kv_decode", args, keep_alive=(lay,))
+
+
+def prepare_prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
+                                 eps, conv_state, slot_mapping, k_data, k_scale, v_data,
+                                 v_scale, state_indices=None, err_flag=None, stream=None):
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    lay = _mx_layout(k_data, k_scale, v_data, v_scale)
+    W = conv_w_k.shape[0]
+    H, D = k_data.shape[2], k_data.shape[3]
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    args = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+            _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
+            ctypes.c_float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
+            _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
+            _ptr(v_data), _ptr(v_scale), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    return PreparedCall("sconv_kv_prefill_varlen_mxfp8", args, keep_alive=(lay,))
+
+
+def prepare_decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
+                         slot_mapping, k_data, k_scale, v_data, v_scale, state_indices=None,
+                         err_flag=None, stream=None):
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    lay = _mx_layout(k_data, k_scale, v_data, v_scale)
+    W = conv_w_k.shape[0]
+    H, D = k_data.shape[2], k_data.shape[3]
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    args = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+            _ptr(gamma_v), ctypes.c_float(eps), W, H, D,
+            _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
+            _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale),
+            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    return PreparedCall("sconv_kv_decode_mxfp8", args, keep_alive=(lay,))

@@ -37,7 +37,14 @@ struct StepParams {
   int64_t stride_head;
   int slot_linear;  // stride_page == page_size * stride_slot
   int* err;
-  int tile;  // tokens per CTA tile (prefill)
+  int tile;  // unused
+  // MXFP8 store (block-scaled): E4M3 data caches (uint8, same element
+  // offsets as the bf16 caches) and E8M0 scale caches (one byte per 32
+  // channels: element offset / 32)
+  uint8_t* k_data;
+  uint8_t* v_data;
+  uint8_t* k_scale;
+  uint8_t* v_scale;
 };
 
 // Flag bits (same values as the public SCONV_KV_FLAG_*).
@@ -110,6 +117,60 @@ __device__ __forceinline__ int64_t slot_row_offset(const StepParams& P,
   if (P.slot_linear) return slot * P.stride_slot;
   const int64_t page = slot / P.page_size;
   return page * P.stride_page + (slot - page * P.page_size) * P.stride_slot;
+}
+
+// ---- MXFP8 (OCP Microscaling) block store: 32 channels = 4 lanes x 8.
+
+// Shared exponent of a block with largest magnitude `amax` (binary32):
+// floor(log2(amax)) - 8, the 8 being the exponent of E4M3's largest normal
+// (448 = 1.75 * 2^8); blocks whose amax is zero or subnormal take -127.
+__device__ __forceinline__ int mx_shared_exponent(float amax) {
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);  // biased
+  return e == 0 ? -127 : max(e - 127 - 8, -127);
+}
+
+// Two binary32 -> two E4M3 codes (nearest even, saturating), low element
+// in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  unsigned short h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+  return h;
+}
+
+// Quantise this lane's 8 normalised values z = t * r (t = conv output times
+// gamma, r = the head's 1/rms; channels d0..d0+7 of a head) as part of their
+// 32-channel block and store: 8 code bytes at `data`, and (lane % 4 == 0
+// of the block's 4 lanes) the E8M0 scale byte at `scale`.  z is formed
+// first and then scaled by the exact power of two 2^-s (<= 2^127, and
+// |z| * 2^-s < 512, so nothing overflows; folding 2^-s into r instead would
+// overflow for all-zero blocks).  All 32 lanes of the warp must call it
+// (shuffles); `write` masks the stores.
+__device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool write,
+                                          uint8_t* data, uint8_t* scale) {
+  const float2 rr = make_float2(r, r);
+  const float2 z[4] = {__fmul2_rn(t[0], rr), __fmul2_rn(t[1], rr), __fmul2_rn(t[2], rr),
+                       __fmul2_rn(t[3], rr)};
+  float amax = fmaxf(fmaxf(fabsf(z[0].x), fabsf(z[0].y)), fmaxf(fabsf(z[1].x), fabsf(z[1].y)));
+  amax = fmaxf(amax, fmaxf(fmaxf(fabsf(z[2].x), fabsf(z[2].y)), fmaxf(fabsf(z[3].x), fabsf(z[3].y))));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+  const int s = mx_shared_exponent(amax);
+  const float m = __uint_as_float(static_cast<uint32_t>(127 - s) << 23);  // 2^-s, exact
+  const float2 mm = make_float2(m, m);
+  const float2 a = __fmul2_rn(z[0], mm), b = __fmul2_rn(z[1], mm);
+  const float2 c = __fmul2_rn(z[2], mm), d = __fmul2_rn(z[3], mm);
+  const uint32_t w0 = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+  const uint32_t w1 = e4m3x2(c.x, c.y) | (e4m3x2(d.x, d.y) << 16);
+  const bool scale_writer = write && ((threadIdx.x & 3) == 0);
+  asm volatile(
+      "{\n\t.reg .pred q, r;\n\t"
+      "setp.ne.b32 q, %0, 0;\n\t"
+      "setp.ne.b32 r, %1, 0;\n\t"
+      "@q st.global.cs.v2.u32 [%2], {%3, %4};\n\t"
+      "@r st.global.cs.u8 [%5], %6;\n\t}" ::"r"(static_cast<int>(write)),
+      "r"(static_cast<int>(scale_writer)), "l"(data), "r"(w0), "r"(w1), "l"(scale),
+      "r"(static_cast<uint32_t>(s + 127))
+      : "memory");
 }
 
 // Hardware reciprocal square root (PTX rsqrt.approx.ftz.f32, one MUFU op;

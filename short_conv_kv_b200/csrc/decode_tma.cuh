@@ -58,7 +58,7 @@ __device__ __forceinline__ void bulk_wait_all() {
 template <int W>
 constexpr int decode_ctas_per_sm() { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
 
-template <int W, int D>
+template <int W, int D, bool MX>
 __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     decode_tma_kernel(const StepParams P, const DecGeom Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -188,7 +188,10 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
   const bool isv = g >= half;
   const int c0 = (isv ? g - half : g) * 8;
   const int d0 = c0 % D;
-  uint16_t* cache = (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  uint16_t* cache = MX ? nullptr : (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  const int64_t head_off = (c0 / D) * P.stride_head + d0;
+  uint8_t* mxdata = MX ? (isv ? P.v_data : P.k_data) + head_off : nullptr;
+  uint8_t* mxscale = MX ? (isv ? P.v_scale : P.k_scale) + (head_off >> 5) : nullptr;
   // taps kept packed (bf16) and widened at use: one token per sequence
   // makes the extra unpacking cheap, and the saved registers buy occupancy
   const uint16_t* w = (isv ? P.w_v : P.w_k) + c0;
@@ -228,7 +231,17 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
       const float ss = group_sum<G>(s2.x + s2.y);
       const float rn = rsqrt_approx(fmaf(ss, P.inv_d, P.eps));
       const long long off = s_off[q];
-      if (active && off >= 0) {
+      if constexpr (MX) {
+        // all lanes take part (the block scale is a 4-lane reduction)
+        const float4 ga = __ldg(reinterpret_cast<const float4*>(gam));
+        const float4 gb = __ldg(reinterpret_cast<const float4*>(gam) + 1);
+        const float2 t[4] = {fmul2(acc[0], make_float2(ga.x, ga.y)),
+                             fmul2(acc[1], make_float2(ga.z, ga.w)),
+                             fmul2(acc[2], make_float2(gb.x, gb.y)),
+                             fmul2(acc[3], make_float2(gb.z, gb.w))};
+        mx_store8(t, rn, active && off >= 0, mxdata + (off >= 0 ? off : 0),
+                  mxscale + (off >= 0 ? (off >> 5) : 0));
+      } else if (active && off >= 0) {
         const float4 ga = __ldg(reinterpret_cast<const float4*>(gam));
         const float4 gb = __ldg(reinterpret_cast<const float4*>(gam) + 1);
         const float2 gm[4] = {make_float2(ga.x, ga.y), make_float2(ga.z, ga.w),

@@ -50,6 +50,9 @@ namespace sconv {
 #ifndef SCONV_PREFILL_EARLY_RELEASE
 #define SCONV_PREFILL_EARLY_RELEASE 0  // copy a stage to registers, then release it
 #endif
+#ifndef SCONV_PREFILL_MX_UNROLL
+#define SCONV_PREFILL_MX_UNROLL 2  // fast-path unroll of the MXFP8 store for W <= 4
+#endif
 #ifndef SCONV_PREFILL_LAST_WARP_REFILL
 #define SCONV_PREFILL_LAST_WARP_REFILL 0  // the last warp to release a stage refills it
 #endif
@@ -63,8 +66,10 @@ constexpr int kTmaRows = SCONV_PREFILL_ROWS;  // token rows per stage
 // CTA per SM with room for an 8-token unroll and gamma in registers.
 template <int W>
 __host__ __device__ constexpr bool gamma_in_smem() { return W <= 4; }
-template <int W>
-__host__ __device__ constexpr int fast_unroll() { return W <= 4 ? 4 : 8; }
+template <int W, bool MX>
+__host__ __device__ constexpr int fast_unroll() {
+  return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : 4) : 8;
+}
 constexpr int kTmaRingBytes2 = SCONV_PREFILL_RING_KB * 1024;
 constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memory
 constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 8;  // per-warp slot offsets
@@ -123,11 +128,13 @@ __device__ __forceinline__ void lds_gamma(const float* g, float2 (&gm)[4]) {
   gm[3] = make_float2(b.z, b.w);
 }
 
-// RMSNorm of the head (D/8 lanes), gamma, bf16 rounding, 16-byte store.
-template <int D>
+// RMSNorm of the head (D/8 lanes), gamma, then either bf16 rounding and a
+// 16-byte store into the bf16 cache (MX = false), or the MXFP8 block store
+// (8 E4M3 bytes + the block's E8M0 scale).
+template <int D, bool MX>
 __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 (&gm)[4],
                                            float inv_d, float eps, bool write,
-                                           uint16_t* dst) {
+                                           uint16_t* dst, uint8_t* mx_data, uint8_t* mx_scale) {
   float2 s2 = fmul2(acc[0], acc[0]);
   s2 = ffma2(acc[1], acc[1], s2);
   s2 = ffma2(acc[2], acc[2], s2);
@@ -135,15 +142,21 @@ __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 
   const float ss = group_sum<D / 8>(s2.x + s2.y);
   const float rn = rsqrt_approx(fmaf(ss, inv_d, eps));
   const float2 rr = make_float2(rn, rn);
-  uint4 o;
-  o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
-  o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
-  o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
-  o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
-  st_stream_if(write, dst, o);
+  if constexpr (MX) {
+    const float2 t[4] = {fmul2(acc[0], gm[0]), fmul2(acc[1], gm[1]), fmul2(acc[2], gm[2]),
+                         fmul2(acc[3], gm[3])};
+    mx_store8(t, rn, write, mx_data, mx_scale);
+  } else {
+    uint4 o;
+    o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
+    o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
+    o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
+    o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
+    st_stream_if(write, dst, o);
+  }
 }
 
-template <int W, int D, int MINB>
+template <int W, int D, int MINB, bool MX>
 __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -273,7 +286,11 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   const int c0 = (isv ? g - half : g) * 8;
   const int d0 = c0 % D;
   const uint16_t* xbase = (isv ? P.v : P.k) + c0;
-  uint16_t* cache = (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  uint16_t* cache = MX ? nullptr : (isv ? P.v_cache : P.k_cache) + (c0 / D) * P.stride_head + d0;
+  // MXFP8 store: element offsets as for bf16 (bytes), scale offset / 32
+  const int64_t head_off = (c0 / D) * P.stride_head + d0;
+  uint8_t* mxdata = MX ? (isv ? P.v_data : P.k_data) + head_off : nullptr;
+  uint8_t* mxscale = MX ? (isv ? P.v_scale : P.k_scale) + (head_off >> 5) : nullptr;
   const int64_t srow = 2 * static_cast<int64_t>(P.C);
   const int st_chan = (isv ? P.C : 0) + c0;
 
@@ -388,15 +405,17 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   }
 
   const float eps = P.eps, inv_d = P.inv_d;
-#define NORM_STORE(pred)                                              \
-  do {                                                                \
-    if constexpr (gamma_in_smem<W>()) {                               \
-      float2 gs[4];                                                   \
-      lds_gamma(my_gamma, gs);                                        \
-      norm_store<D>(acc, gs, inv_d, eps, (pred), cache + off);        \
-    } else {                                                          \
-      norm_store<D>(acc, gm, inv_d, eps, (pred), cache + off);        \
-    }                                                                 \
+#define NORM_STORE(pred)                                                            \
+  do {                                                                              \
+    uint8_t* mxd = MX ? mxdata + off : nullptr;                                     \
+    uint8_t* mxs = MX ? mxscale + (off >> 5) : nullptr;                             \
+    if constexpr (gamma_in_smem<W>()) {                                             \
+      float2 gs[4];                                                                 \
+      lds_gamma(my_gamma, gs);                                                      \
+      norm_store<D, MX>(acc, gs, inv_d, eps, (pred), cache + off, mxd, mxs);        \
+    } else {                                                                        \
+      norm_store<D, MX>(acc, gm, inv_d, eps, (pred), cache + off, mxd, mxs);        \
+    }                                                                               \
   } while (0)
   // inactive lanes read column 0 (and never store): no predicated loads
   const unsigned char* my_ring = ring + (active ? lg : 0) * 16;
@@ -450,7 +469,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
         NORM_STORE(active && r < rows && off >= 0);
       }
 #else
-#pragma unroll fast_unroll<W>()
+#pragma unroll fast_unroll<W, MX>()
       for (int r = 0; r < R; ++r) {
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
         float2 acc[4];

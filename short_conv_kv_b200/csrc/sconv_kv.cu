@@ -26,12 +26,7 @@ using TmaFn = void (*)(StepParams, sconv::TmaGeom);
 template <int W>
 constexpr int prefill_ctas_per_sm() { return W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1; }
 
-template <int W, int D>
-TmaFn prefill_fn() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>()>; }
 using DecFn = void (*)(StepParams, sconv::DecGeom);
-
-template <int W, int D>
-DecFn decode_fn() { return sconv::decode_tma_kernel<W, D>; }
 
 // Kernel instance for (W, D): F<W, D>() over W in 1..8, D in {64, 128, 256}.
 template <typename Fn, template <int, int> class F>
@@ -59,13 +54,22 @@ struct Pick {
     }
   }
 };
+// bf16 store / MXFP8 store instances of each kernel
 template <int W, int D>
 struct DecodeK {
-  static DecFn get() { return decode_fn<W, D>(); }
+  static DecFn get() { return sconv::decode_tma_kernel<W, D, false>; }
+};
+template <int W, int D>
+struct DecodeKMx {
+  static DecFn get() { return sconv::decode_tma_kernel<W, D, true>; }
 };
 template <int W, int D>
 struct PrefillK {
-  static TmaFn get() { return prefill_fn<W, D>(); }
+  static TmaFn get() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), false>; }
+};
+template <int W, int D>
+struct PrefillKMx {
+  static TmaFn get() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), true>; }
 };
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -114,10 +118,12 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
                     int num_kv_heads, int head_dim, void* conv_state,
                     int64_t state_pool_size, const int64_t* slot_mapping,
                     void* k_cache, void* v_cache,
-                    const sconv_kv_cache_layout_t* layout, StepParams* P) {
+                    const sconv_kv_cache_layout_t* layout, StepParams* P,
+                    uint8_t* k_scale = nullptr, uint8_t* v_scale = nullptr, bool mx = false) {
   if (!k || !v || !conv_w_k || !conv_w_v || !gamma_k || !gamma_v ||
       !slot_mapping || !k_cache || !v_cache || !layout)
     return SCONV_KV_ERR_NULL;
+  if (mx && (!k_scale || !v_scale)) return SCONV_KV_ERR_NULL;
   if (W > 1 && !conv_state) return SCONV_KV_ERR_NULL;
   if (W < 1 || W > SCONV_KV_MAX_W) return SCONV_KV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return SCONV_KV_ERR_SHAPE;
@@ -136,6 +142,9 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
       !aligned16(v_cache) || (conv_state && !aligned16(conv_state)))
     return SCONV_KV_ERR_ALIGN;
   if (layout->stride_head % 8 || layout->stride_slot % 8 || layout->stride_page % 8)
+    return SCONV_KV_ERR_ALIGN;
+  // MXFP8: a scale byte per 32 elements, so element strides are multiples of 32
+  if (mx && (layout->stride_head % 32 || layout->stride_slot % 32 || layout->stride_page % 32))
     return SCONV_KV_ERR_ALIGN;
 
   memset(P, 0, sizeof(*P));
@@ -160,6 +169,14 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
   P->stride_slot = layout->stride_slot;
   P->stride_head = layout->stride_head;
   P->slot_linear = layout->stride_page == layout->page_size * layout->stride_slot;
+  if (mx) {
+    P->k_data = static_cast<uint8_t*>(k_cache);
+    P->v_data = static_cast<uint8_t*>(v_cache);
+    P->k_scale = k_scale;
+    P->v_scale = v_scale;
+    P->k_cache = nullptr;
+    P->v_cache = nullptr;
+  }
   return SCONV_KV_OK;
 }
 
@@ -189,50 +206,15 @@ int launch(const void* fn, dim3 grid, dim3 block, void** args, size_t smem, void
 }
 
 
-}  // namespace
-
-extern "C" {
-
-int sconv_kv_version(void) { return 100; }
-
-const char* sconv_kv_strerror(int status) {
-  switch (status) {
-    case SCONV_KV_OK: return "ok";
-    case SCONV_KV_ERR_NULL: return "a required pointer is NULL";
-    case SCONV_KV_ERR_SHAPE: return "bad shape (W, head_dim, heads, counts, strides or layout)";
-    case SCONV_KV_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
-    case SCONV_KV_ERR_UNSUPPORTED: return "unsupported combination";
-    case SCONV_KV_ERR_CUDA: return "CUDA error at launch (see sconv_kv_last_cuda_error)";
-    default: return "unknown status";
-  }
-}
-
-const char* sconv_kv_last_cuda_error(void) { return g_cuda_error; }
-
-int sconv_kv_cache_layout(int64_t num_pages, int64_t page_size, int num_kv_heads,
-                          int head_dim, sconv_kv_cache_layout_t* out) {
-  if (!out) return SCONV_KV_ERR_NULL;
-  if (num_pages < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1)
-    return SCONV_KV_ERR_SHAPE;
-  out->num_pages = num_pages;
-  out->page_size = page_size;
-  out->num_kv_heads = num_kv_heads;
-  out->head_dim = head_dim;
-  out->stride_head = head_dim;
-  out->stride_slot = static_cast<int64_t>(num_kv_heads) * head_dim;
-  out->stride_page = page_size * out->stride_slot;
-  out->bytes_per_cache = num_pages * out->stride_page * 2;
-  return SCONV_KV_OK;
-}
-
-int sconv_kv_prefill_varlen(
+int prefill_impl(
     const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
     const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
     const void* conv_w_v, const float* gamma_k, const float* gamma_v,
     float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
     const int32_t* state_indices, int64_t state_pool_size,
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
-    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream, bool mx,
+    uint8_t* k_scale, uint8_t* v_scale) {
   // an empty call enqueues nothing; its pointers are not examined (empty
   // tensors may have NULL data pointers)
   if (num_seqs < 0 || num_tokens < 0 || num_tokens > INT32_MAX) return SCONV_KV_ERR_SHAPE;
@@ -240,10 +222,10 @@ int sconv_kv_prefill_varlen(
   StepParams P;
   int rc = validate_common(k, v, row_stride, conv_w_k, conv_w_v, gamma_k, gamma_v, W,
                            num_kv_heads, head_dim, conv_state, state_pool_size,
-                           slot_mapping, k_cache, v_cache, layout, &P);
+                           slot_mapping, k_cache, v_cache, layout, &P, k_scale, v_scale, mx);
   if (rc != SCONV_KV_OK) return rc;
   if (!cu_seqlens) return SCONV_KV_ERR_NULL;
-  TmaFn fn = Pick<TmaFn, PrefillK>::get(W, head_dim);
+  TmaFn fn = mx ? Pick<TmaFn, PrefillKMx>::get(W, head_dim) : Pick<TmaFn, PrefillK>::get(W, head_dim);
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
 
   P.num_tokens = num_tokens;
@@ -290,21 +272,21 @@ int sconv_kv_prefill_varlen(
                 stream);
 }
 
-int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
-                    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
-                    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
-                    void* conv_state, const int32_t* state_indices,
-                    int64_t state_pool_size, const int64_t* slot_mapping, void* k_cache,
-                    void* v_cache, const sconv_kv_cache_layout_t* layout, int* err_flag,
-                    void* stream) {
+int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
+                const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+                const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+                void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
+                const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream, bool mx,
+                uint8_t* k_scale, uint8_t* v_scale) {
   if (batch < 0) return SCONV_KV_ERR_SHAPE;
   if (batch == 0) return SCONV_KV_OK;  // nothing enqueued, pointers not examined
   StepParams P;
   int rc = validate_common(k, v, row_stride, conv_w_k, conv_w_v, gamma_k, gamma_v, W,
                            num_kv_heads, head_dim, conv_state, state_pool_size,
-                           slot_mapping, k_cache, v_cache, layout, &P);
+                           slot_mapping, k_cache, v_cache, layout, &P, k_scale, v_scale, mx);
   if (rc != SCONV_KV_OK) return rc;
-  DecFn fn = Pick<DecFn, DecodeK>::get(W, head_dim);
+  DecFn fn = mx ? Pick<DecFn, DecodeKMx>::get(W, head_dim) : Pick<DecFn, DecodeK>::get(W, head_dim);
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
   P.num_tokens = batch;
   P.num_seqs = batch;
@@ -342,6 +324,96 @@ int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
   void* args[] = {&P, &G};
   return launch(reinterpret_cast<const void*>(fn), dim3(G.ctas, ctas_y), block, args, smem,
                 stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int sconv_kv_version(void) { return 100; }
+
+const char* sconv_kv_strerror(int status) {
+  switch (status) {
+    case SCONV_KV_OK: return "ok";
+    case SCONV_KV_ERR_NULL: return "a required pointer is NULL";
+    case SCONV_KV_ERR_SHAPE: return "bad shape (W, head_dim, heads, counts, strides or layout)";
+    case SCONV_KV_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case SCONV_KV_ERR_UNSUPPORTED: return "unsupported combination";
+    case SCONV_KV_ERR_CUDA: return "CUDA error at launch (see sconv_kv_last_cuda_error)";
+    default: return "unknown status";
+  }
+}
+
+const char* sconv_kv_last_cuda_error(void) { return g_cuda_error; }
+
+int sconv_kv_cache_layout(int64_t num_pages, int64_t page_size, int num_kv_heads,
+                          int head_dim, sconv_kv_cache_layout_t* out) {
+  if (!out) return SCONV_KV_ERR_NULL;
+  if (num_pages < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1)
+    return SCONV_KV_ERR_SHAPE;
+  out->num_pages = num_pages;
+  out->page_size = page_size;
+  out->num_kv_heads = num_kv_heads;
+  out->head_dim = head_dim;
+  out->stride_head = head_dim;
+  out->stride_slot = static_cast<int64_t>(num_kv_heads) * head_dim;
+  out->stride_page = page_size * out->stride_slot;
+  out->bytes_per_cache = num_pages * out->stride_page * 2;
+  return SCONV_KV_OK;
+}
+
+int sconv_kv_prefill_varlen(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                      gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
+                      state_indices, state_pool_size, slot_mapping, k_cache, v_cache, layout,
+                      err_flag, stream, false, nullptr, nullptr);
+}
+
+int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
+                    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+                    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+                    void* conv_state, const int32_t* state_indices,
+                    int64_t state_pool_size, const int64_t* slot_mapping, void* k_cache,
+                    void* v_cache, const sconv_kv_cache_layout_t* layout, int* err_flag,
+                    void* stream) {
+  return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
+                     num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
+                     slot_mapping, k_cache, v_cache, layout, err_flag, stream, false, nullptr,
+                     nullptr);
+}
+
+int sconv_kv_prefill_varlen_mxfp8(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                      gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
+                      state_indices, state_pool_size, slot_mapping, k_data, v_data, layout,
+                      err_flag, stream, true, k_scale, v_scale);
+}
+
+int sconv_kv_decode_mxfp8(const void* k, const void* v, int64_t row_stride, int batch,
+                          const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+                          const float* gamma_v, float eps, int W, int num_kv_heads,
+                          int head_dim, void* conv_state, const int32_t* state_indices,
+                          int64_t state_pool_size, const int64_t* slot_mapping, void* k_data,
+                          uint8_t* k_scale, void* v_data, uint8_t* v_scale,
+                          const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
+                     num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
+                     slot_mapping, k_data, v_data, layout, err_flag, stream, true, k_scale,
+                     v_scale);
 }
 
 }  // extern "C"

@@ -175,3 +175,99 @@ def expected_final_state(k_bits, v_bits, cu, state_bits, W, state_indices=None):
             else:
                 st[si, j] = old[W - 1 + q]
     return st
+
+
+# ------------------------------------------------------------------ MXFP8 store
+
+MX_SENTINEL = 0xFF
+
+
+def check_mx(gpu_data, gpu_scale, slot_mapping, z, what=""):
+    """GPU MXFP8 caches (uint8 data [P, S, H, D], scales [P, S, H, D/32])
+    against the oracle's unrounded z [T, H*D] (double).
+
+    Decisions are taken on z rounded to binary32 on both sides; the GPU's
+    binary32 z may differ from the oracle's by a few ulps, so:
+      - a block scale must equal the oracle's, or differ by one when the
+        block's amax lies within 1e-5 (relative) of the power of two where
+        the scale steps;
+      - every element code must be the E4M3 rounding of z / 2^s under the
+        GPU's scale s, except an adjacent code when z / 2^s lies within
+        fp32 evaluation error of the midpoint between the two;
+      - slots not in slot_mapping keep the sentinel bytes.
+    """
+    P, S, H, D = gpu_data.shape
+    NB = D // 32
+    gd = gpu_data.reshape(P * S, H, D)
+    gs = gpu_scale.reshape(P * S, H, NB)
+    sm = np.asarray(slot_mapping)
+    tok = np.nonzero(sm >= 0)[0]
+    written = np.zeros(P * S, bool)
+    written[sm[tok]] = True
+    assert np.all(gd[~written] == MX_SENTINEL), f"{what}: untouched data changed"
+    assert np.all(gs[~written] == MX_SENTINEL), f"{what}: untouched scales changed"
+    if tok.size == 0:
+        return {}
+    zf = np.asarray(z, np.float64)[tok].astype(np.float32).astype(np.float64).reshape(-1, H, NB, 32)
+    g_codes = gd[sm[tok]].reshape(-1, H, NB, 32)
+    s_g = gs[sm[tok]].astype(np.int64) - 127
+    amax = np.abs(zf).max(axis=-1)
+    _, e = np.frexp(amax)
+    s_o = np.where(amax < 2.0 ** -126, -127, np.clip(e - 1 - 8, -127, 127))
+    bad_scale = s_g != s_o
+    if bad_scale.any():
+        edge = 2.0 ** (np.maximum(s_g, s_o) + 8).astype(np.float64)
+        near = (np.abs(s_g - s_o) == 1) & (np.abs(amax - edge) <= 1e-5 * edge)
+        assert np.all(near[bad_scale]), (
+            f"{what}: {int((bad_scale & ~near).sum())} block scales differ away from a "
+            f"power-of-two boundary")
+    u = zf * np.exp2(-s_g.astype(np.float64))[..., None]
+    exp_codes = oracle.e4m3_from_f64(u)
+    mism = g_codes != exp_codes
+    if mism.any():
+        gv = oracle.e4m3_to_f64(g_codes[mism])
+        ev = oracle.e4m3_to_f64(exp_codes[mism])
+        uu = u[mism]
+        gc = g_codes[mism].astype(np.int64)
+        ec = exp_codes[mism].astype(np.int64)
+        adjacent = ((gc & 0x80) == (ec & 0x80)) & (np.abs((gc & 0x7F) - (ec & 0x7F)) == 1)
+        tiny = (np.abs(gv) <= 2.0 ** -9) & (np.abs(ev) <= 2.0 ** -9)
+        scale_mag = np.exp2(-np.broadcast_to(s_g[..., None], u.shape)[mism].astype(np.float64))
+        margin = 2e-5 * np.abs(uu) + 1e-6 * scale_mag
+        near_tie = np.abs(uu - 0.5 * (gv + ev)) <= margin
+        ok = (adjacent | tiny) & near_tie
+        assert ok.all(), (f"{what}: {int((~ok).sum())} element codes differ from the E4M3 "
+                          f"rounding away from a tie; e.g. u={uu[~ok][:4]}, gpu={gv[~ok][:4]}, "
+                          f"rne={ev[~ok][:4]}")
+    return dict(scale_mismatch=float(bad_scale.mean()), code_mismatch=float(mism.mean()))
+
+
+def mx_caches(num_pages, page_size, H, D, device="cuda"):
+    """Sentinel-filled MXFP8 data and scale caches."""
+    data = torch.full((num_pages, page_size, H, D), MX_SENTINEL, dtype=torch.uint8, device=device)
+    scale = torch.full((num_pages, page_size, H, D // 32), MX_SENTINEL, dtype=torch.uint8,
+                       device=device)
+    return data, scale
+
+
+def run_gpu_prefill_mx(b: wl.Batch, state=None, err=None):
+    from short_conv_kv_b200 import binding
+    kd, ks = mx_caches(b.num_pages, b.page_size, b.Hkv, b.D)
+    vd, vs = mx_caches(b.num_pages, b.page_size, b.Hkv, b.D)
+    st = dev(b.conv_state.clone()) if state is None else state
+    binding.prefill_varlen_mxfp8(
+        dev(b.k), dev(b.v), dev(b.cu_seqlens), dev(b.conv_w_k), dev(b.conv_w_v),
+        dev(b.gamma_k), dev(b.gamma_v), b.eps, st, dev(b.slot_mapping), kd, ks, vd, vs,
+        state_indices=dev(b.state_indices), err_flag=err)
+    torch.cuda.synchronize()
+    return kd, ks, vd, vs, st
+
+
+def full_parity_mx(b: wl.Batch):
+    kd, ks, vd, vs, st = run_gpu_prefill_mx(b)
+    ref = oracle_prefill(b)
+    sm = b.slot_mapping.numpy()
+    rk = check_mx(kd.cpu().numpy(), ks.cpu().numpy(), sm, ref["z_k"], "k mx")
+    rv = check_mx(vd.cpu().numpy(), vs.cpu().numpy(), sm, ref["z_v"], "v mx")
+    assert np.array_equal(wl.bits(st.cpu()), ref["conv_state"]), "conv_state differs"
+    return rk, rv
