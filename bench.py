@@ -47,12 +47,14 @@ KERNEL_SOURCES = [os.path.join(ROOT, "short_conv_kv_b200", "csrc", f)
 
 # ------------------------------------------------------------------ helpers
 
-def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8):
+def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8, mx=False):
     """Bytes the step must move: per token K+V rows in and K+V cache rows out
-    plus the slot; per sequence the conv_state rows in and out; per launch
-    the taps and gammas."""
+    (bf16, or with the MXFP8 store one E4M3 byte per channel plus one scale
+    byte per 32 channels) plus the slot; per sequence the conv_state rows in
+    and out; per launch the taps and gammas."""
     C = Hkv * D
-    per_token = 2 * C * 2 + 2 * C * 2 + slot_bytes
+    out = 2 * C + 2 * C // 32 if mx else 2 * C * 2
+    per_token = 2 * C * 2 + out + slot_bytes
     per_seq = 2 * (W - 1) * 2 * C * 2
     per_launch = 2 * W * C * 2 + 2 * D * 4
     return tokens * per_token + seqs * per_seq + per_launch
@@ -157,6 +159,8 @@ class Workload:
     """Device-resident rotating input sets plus host copies for e2e."""
 
     def __init__(self, name, rank):
+        self.mx = name.endswith("_mx")  # MXFP8 cache store variant
+        name = name[:-3] if self.mx else name
         self.name, self.rank = name, rank
         seed_shift = 97 * rank
         if name == "single":
@@ -192,7 +196,8 @@ class Workload:
             b = self.batches[0]
             self.W, self.Hkv, self.D = b.W, b.Hkv, b.D
             self.tokens_per_step, self.seqs_per_step = b.num_tokens, b.num_seqs
-            self.bytes_per_step = algorithmic_bytes(b.num_tokens, b.num_seqs, b.W, b.Hkv, b.D)
+            self.bytes_per_step = algorithmic_bytes(b.num_tokens, b.num_seqs, b.W, b.Hkv, b.D,
+                                                    mx=self.mx)
             shared = dict(conv_w_k=b.conv_w_k.to(dev), conv_w_v=b.conv_w_v.to(dev),
                           gamma_k=b.gamma_k.to(dev), gamma_v=b.gamma_v.to(dev))
             R = max(1, math.ceil(3 * L2_BYTES / self.bytes_per_step))
@@ -207,7 +212,7 @@ class Workload:
             s = self.long
             self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
             self.tokens_per_step, self.seqs_per_step = s.chunk, 1
-            self.bytes_per_step = algorithmic_bytes(s.chunk, 1, s.W, s.Hkv, s.D)
+            self.bytes_per_step = algorithmic_bytes(s.chunk, 1, s.W, s.Hkv, s.D, mx=self.mx)
             shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
                           gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
                           conv_state=s.initial_state().to(dev),
@@ -221,7 +226,7 @@ class Workload:
             s = self.dec
             self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
             self.tokens_per_step, self.seqs_per_step = s.batch, s.batch
-            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D)
+            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D, mx=self.mx)
             shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
                           gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
                           k_cache=s.empty_cache().to(dev), v_cache=s.empty_cache().to(dev))
@@ -233,8 +238,33 @@ class Workload:
                 self.calls_args.append(dict(k=k.to(dev), v=v.to(dev), slot_mapping=sm.to(dev),
                                             conv_state=states[r % len(states)], **shared))
 
+        if self.mx:
+            # MXFP8 store: uint8 E4M3 data + E8M0 scale caches in place of
+            # the bf16 caches (one set per distinct bf16 cache)
+            made = {}
+            for a in self.calls_args:
+                for key in ("k_cache", "v_cache"):
+                    c = a.pop(key)
+                    if id(c) not in made:
+                        P_, S_, H_, D_ = c.shape
+                        made[id(c)] = (
+                            torch.full((P_, S_, H_, D_), 0xFF, dtype=torch.uint8, device=dev),
+                            torch.full((P_, S_, H_, D_ // 32), 0xFF, dtype=torch.uint8, device=dev))
+                    a[key[0] + "_data"], a[key[0] + "_scale"] = made[id(c)]
+            self.desc += "; MXFP8 cache store (E4M3 + E8M0 per 32 channels)"
+
     def prepared(self, i, stream):
         a = self.calls_args[i % len(self.calls_args)]
+        if self.mx and self.kind == "decode":
+            return self.binding.prepare_decode_mxfp8(
+                a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
+                a["eps"], a["conv_state"], a["slot_mapping"], a["k_data"], a["k_scale"],
+                a["v_data"], a["v_scale"], stream=stream)
+        if self.mx:
+            return self.binding.prepare_prefill_varlen_mxfp8(
+                a["k"], a["v"], a["cu_seqlens"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"],
+                a["gamma_v"], a["eps"], a["conv_state"], a["slot_mapping"], a["k_data"],
+                a["k_scale"], a["v_data"], a["v_scale"], stream=stream)
         if self.kind == "decode":
             return self.binding.prepare_decode(
                 a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
@@ -246,8 +276,105 @@ class Workload:
             a["v_cache"], stream=stream)
 
     def kernel_tag(self):
-        return {"prefill": "prefill_tma_kernel", "long": "prefill_tma_kernel",
-                "decode": "decode_tma_kernel"}[self.kind]
+        tag = {"prefill": "prefill_tma_kernel", "long": "prefill_tma_kernel",
+               "decode": "decode_tma_kernel"}[self.kind]
+        return tag + ("_mx" if self.mx else "")
+
+
+# ------------------------------------------------------------------ unfused chain
+
+class UnfusedChain:
+    """Bench-only context for the fusion claim ("SGLang and Miles announce
+    day-0 Inkling support", aib.vote English news item, paragraph 2: the
+    fused K/V conv + normalisation + KV-cache write against an unfused
+    chain): the same step as a chain of stock torch ops, each one writing
+    its intermediate to HBM.
+
+      1. gather: per sequence, its W-1 state rows then its tokens' K|V rows
+         into one bf16 buffer `xcat` (index_copy_);
+      2. conv: acc[r] = sum_j w[j] * xcat[r + j] in fp32 (W passes);
+      3. pick each token's conv row, per-head RMSNorm (F.rms_norm), times
+         gamma, round to bf16;
+      4. cache write: index_copy_ of the K and V rows into the paged caches;
+      5. state update: the last W-1 rows of each sequence's segment of
+         `xcat` copied back into its state row.
+
+    Identity state indices, every slot >= 0 (as in the bench workloads).
+    Not the product: nothing here is on the library's path."""
+
+    def __init__(self, lengths, W, Hkv, D, dev):
+        import numpy as np_
+        self.W, self.Hkv, self.D, self.C = W, Hkv, D, Hkv * D
+        Wm = W - 1
+        lengths = [int(x) for x in lengths]
+        self.S, self.T = len(lengths), sum(lengths)
+        seg = np_.cumsum([0] + [Wm + L for L in lengths])
+        tok = np_.concatenate([seg[i] + Wm + np_.arange(L) for i, L in enumerate(lengths)]
+                              + [np_.zeros(0, np_.int64)])
+        st = np_.concatenate([seg[i] + np_.arange(Wm) for i in range(self.S)]
+                             + [np_.zeros(0, np_.int64)])
+        new_st = np_.concatenate([seg[i] + L + np_.arange(Wm) for i, L in enumerate(lengths)]
+                                 + [np_.zeros(0, np_.int64)])
+        rows = int(seg[-1])
+        self.N = rows - Wm  # conv rows computed (one per window start)
+        as_t = lambda a: torch.from_numpy(np_.asarray(a, np_.int64)).to(dev)
+        self.tok_pos, self.st_pos, self.new_st = as_t(tok), as_t(st), as_t(new_st)
+        self.out_rows = as_t(tok - Wm)
+        self.xcat = torch.zeros(rows, 2 * self.C, dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, a):
+        T, C, S, Wm, N = self.T, self.C, self.S, self.W - 1, self.N
+        x = torch.cat([a["k"].reshape(T, C), a["v"].reshape(T, C)], dim=1)
+        st = a["conv_state"]
+        self.xcat.index_copy_(0, self.tok_pos, x)
+        if Wm:
+            self.xcat.index_copy_(0, self.st_pos, st[:S].reshape(S * Wm, 2 * C))
+        w = torch.cat([a["conv_w_k"], a["conv_w_v"]], dim=1).float()
+        acc = self.xcat[0:N].float() * w[0]
+        for j in range(1, self.W):
+            acc.addcmul_(self.xcat[j:j + N].float(), w[j])
+        y = acc.index_select(0, self.out_rows).view(T, 2, self.Hkv, self.D)
+        g = torch.stack([a["gamma_k"], a["gamma_v"]]).view(1, 2, 1, self.D)
+        z = (torch.nn.functional.rms_norm(y, (self.D,), eps=a["eps"]) * g).to(torch.bfloat16)
+        sm = a["slot_mapping"]
+        a["k_cache"].view(-1, C).index_copy_(0, sm, z[:, 0].reshape(T, C))
+        a["v_cache"].view(-1, C).index_copy_(0, sm, z[:, 1].reshape(T, C))
+        if Wm:
+            st[:S].copy_(self.xcat.index_select(0, self.new_st).view(S, Wm, 2 * C))
+
+
+def unfused_lengths(work):
+    if work.kind == "prefill":
+        return work.batches[0].cu_seqlens.diff().tolist()
+    if work.kind == "long":
+        return [work.long.chunk]
+    return [1] * work.dec.batch
+
+
+def time_unfused(work, K, Wu, dev):
+    """The unfused chain over the same rotating buffers, K steps in one CUDA
+    graph replay (same method as the fused kernel's timing)."""
+    chain = UnfusedChain(unfused_lengths(work), work.W, work.Hkv, work.D, dev)
+    stream = torch.cuda.Stream(device=dev)
+    n = len(work.calls_args)
+    with torch.cuda.stream(stream):
+        for i in range(Wu):
+            chain(work.calls_args[i % n])
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(K):
+            chain(work.calls_args[i % n])
+    g.replay()
+    torch.cuda.synchronize()
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_ev.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    e_ev.record(stream)
+    e_ev.synchronize()
+    del g
+    return s_ev.elapsed_time(e_ev) / K
 
 
 # ------------------------------------------------------------------ our arm
@@ -471,8 +598,23 @@ def run_ours(args):
     ms_per_step = total_ms / K
     kern_ms = ms_per_step  # one launch per step
     value = world * work.tokens_per_step * K / (total_ms / 1e3)
-    e2e_ms, h2d, d2h = time_e2e(work, args.e2e_steps, dev)
-    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = None
+    if not work.mx:  # the end-to-end leg is measured on the bf16 store
+        e2e_ms, h2d, d2h = time_e2e(work, args.e2e_steps, dev)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e = {"value": world * work.tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "method": "pinned host buffers; upload of the inputs, the step, and download "
+                         "of the written cache rows + new state, pipelined over two buffer "
+                         "sets on three streams"}
+    unfused = None
+    if not work.mx and not args.no_unfused:
+        Ku = min(K, 50)
+        un_ms = max_over_ranks(time_unfused(work, Ku, Wu, dev), world)
+        unfused = {"ms_per_step": un_ms, "steps": Ku, "fused_speedup": un_ms / ms_per_step,
+                   "kind": "bench-only context: the same step as a chain of stock torch ops "
+                           "(gather, fp32 W-tap conv, rms_norm * gamma, bf16, index_copy_ "
+                           "into the caches, state copy), one CUDA graph replay"}
     peaks, peak_src = measured_peaks()
     achieved = work.bytes_per_step / (kern_ms / 1e3) / 1e9
     cpu = None
@@ -484,7 +626,9 @@ def run_ours(args):
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wu,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": work.desc, "storage": "bf16 in, bf16 cache/state, fp32 math",
+            "config": {"workload": work.desc,
+                       "storage": ("bf16 in, MXFP8 cache, bf16 state, fp32 math" if work.mx
+                                   else "bf16 in, bf16 cache/state, fp32 math"),
                        "tokens_per_step_per_gpu": work.tokens_per_step,
                        "seqs_per_step_per_gpu": work.seqs_per_step, "W": work.W,
                        "num_kv_heads": work.Hkv, "head_dim": work.D,
@@ -500,12 +644,8 @@ def run_ours(args):
                          "algorithmic_bytes_per_launch": work.bytes_per_step,
                          "kernel_ms_per_launch": kern_ms},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * work.tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms,
-                    "method": "pinned host buffers; upload of the inputs, the step, and download "
-                              "of the written cache rows + new state, pipelined over two buffer "
-                              "sets on three streams"},
+            "unfused_chain": unfused,
+            "e2e": e2e,
             "gpu_launches": K,
             "clocks": clocks,
         }
@@ -593,9 +733,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="single",
-                    choices=["single", "varlen", "decode", "long", "wsweep2", "wsweep4", "wsweep8"])
+                    choices=["single", "varlen", "decode", "long", "wsweep2", "wsweep4", "wsweep8",
+                             "single_mx", "varlen_mx", "decode_mx", "long_mx"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-unfused", action="store_true",
+                    help="skip timing the unfused torch-op chain (context only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
