@@ -734,7 +734,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="single",
                     choices=["single", "varlen", "decode", "long", "wsweep2", "wsweep4", "wsweep8",
-                             "single_mx", "varlen_mx", "decode_mx", "long_mx"])
+                             "single_mx", "varlen_mx", "decode_mx", "long_mx", "wsweep2_mx",
+                             "wsweep4_mx", "wsweep8_mx"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true",

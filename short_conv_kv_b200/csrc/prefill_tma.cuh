@@ -12,9 +12,10 @@
 //
 // Pipeline.  The rows of the CTA's range (the W-1 rows in front of a range
 // that starts inside a sequence are read directly) stream through a ring of
-// `stages` shared-memory stages of kTmaRows token rows each: one bulk
-// asynchronous copy per row part (K part, V part), completion counted in
-// bytes on the stage's "full" barrier.  Every warp waits on "full", copies
+// `stages` shared-memory stages of kTmaRows token rows each, filled by bulk
+// asynchronous copies (for packed rows, one per chunk for K and one for V;
+// otherwise one per row part), completion counted in bytes on the stage's
+// "full" barrier.  Every warp waits on "full", copies
 // the stage's rows into registers and arrives on the stage's "empty"
 // barrier.  Thread 0 is also the producer: it fills the whole ring up front,
 // and in iteration c it refills the stage of chunk c-1 (once every warp has
@@ -50,8 +51,17 @@ namespace sconv {
 #ifndef SCONV_PREFILL_EARLY_RELEASE
 #define SCONV_PREFILL_EARLY_RELEASE 0  // copy a stage to registers, then release it
 #endif
+#ifndef SCONV_PREFILL_BF16_UNROLL
+#define SCONV_PREFILL_BF16_UNROLL 4  // fast-path unroll of the bf16 store for W <= 4
+#endif
 #ifndef SCONV_PREFILL_MX_UNROLL
 #define SCONV_PREFILL_MX_UNROLL 2  // fast-path unroll of the MXFP8 store for W <= 4
+#endif
+#ifndef SCONV_PREFILL_BLOCK_LAYOUT
+// Stage layout: 1 = [K rows][V rows] (one bulk copy per part when rows are
+// packed), 0 = row by row (one copy per row part), 2 = per instance as
+// block_layout<W, MX>() says.
+#define SCONV_PREFILL_BLOCK_LAYOUT 2
 #endif
 #ifndef SCONV_PREFILL_LAST_WARP_REFILL
 #define SCONV_PREFILL_LAST_WARP_REFILL 0  // the last warp to release a stage refills it
@@ -68,7 +78,16 @@ template <int W>
 __host__ __device__ constexpr bool gamma_in_smem() { return W <= 4; }
 template <int W, bool MX>
 __host__ __device__ constexpr int fast_unroll() {
-  return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : 4) : 8;
+  return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : SCONV_PREFILL_BF16_UNROLL) : 8;
+}
+// Measured on B200: the block layout (2 bulk copies per chunk instead of
+// 2 per row) speeds up the wide-window and MXFP8 instances by 14-25 %; in
+// the W=4 bf16 instance its extra per-thread register spills at the
+// 128-register cap and costs 5 %, so that one keeps the row layout.
+template <int W, bool MX>
+__host__ __device__ constexpr bool block_layout() {
+  return SCONV_PREFILL_BLOCK_LAYOUT == 1 ||
+         (SCONV_PREFILL_BLOCK_LAYOUT == 2 && !(W == 4 && !MX));
 }
 constexpr int kTmaRingBytes2 = SCONV_PREFILL_RING_KB * 1024;
 constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memory
@@ -79,6 +98,8 @@ struct TmaGeom {
   int slice;      // channel groups per full slice (min(NG, 256))
   int stages;     // ring depth
   int ctas;       // persistent CTAs along the token axis
+  int cut_q;      // num_tokens / ctas
+  int cut_r;      // num_tokens % ctas (the first cut_r ranges take one more token)
   int cu_smem;    // cu_seqlens copied to shared memory (num_seqs < kTmaCuSmemMax)
   int smem_ring;  // bytes of the stage ring
   unsigned long long timeout_ns;
@@ -219,7 +240,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   };
   // start of range b: even cut, moved off positions 1..W-2 of a sequence
   auto cut = [&](int b) -> int {
-    int s = static_cast<int>((static_cast<int64_t>(b) * T) / Gm.ctas);
+    int s = b * Gm.cut_q + min(b, Gm.cut_r);
     if (s >= T) return T;
     if (W > 1) {
       const int i = seq_of(s);
@@ -230,9 +251,11 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
     return s;
   };
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    bool ok = cu(0) == 0 && cu(S) == T;
-    for (int i = 0; i < S && ok; ++i) ok = cu(i) <= cu(i + 1);
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    // cu_seqlens must start at 0, end at T and never decrease (the block's
+    // threads check the entries in parallel)
+    bool ok = threadIdx.x != 0 || (cu(0) == 0 && cu(S) == T);
+    for (int i = threadIdx.x; i < S && ok; i += blockDim.x) ok = cu(i) <= cu(i + 1);
     if (!ok) raise_flag(P.err, kFlagCuSeqlens);
   }
   const int ta = cut(blockIdx.x);
@@ -250,17 +273,48 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   // =================================================================== producer
   // Issue chunk c (rows first_row + c*R ...) into stage `st` (= c % NS,
   // tracked by the caller without a division).
+  // Block layout: a stage holds its R rows' K parts (kn*16 bytes each) back
+  // to back, then their V parts.  When a part is a whole row of a packed
+  // tensor (row_stride == C), the chunk's rows of that part are one
+  // contiguous range in global memory and take a single bulk copy.  Row
+  // layout: row r of the stage is its K part then its V part.
+  constexpr bool kBlock = block_layout<W, MX>();
+  const bool k_packed = kn == half && P.row_stride == P.C;
+  const bool v_packed = vn == half && P.row_stride == P.C;
   auto issue = [&](int c, int st) {
     const int r0 = first_row + c * R;
     const int rows = min(R, tb - r0);
     mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(rows * row_bytes));
-    unsigned char* dst = ring + static_cast<size_t>(st) * R * row_bytes;
-    for (int r = 0; r < rows; ++r) {
-      const int64_t t = r0 + r;
-      if (kn) bulk_g2s(dst, P.k + t * P.row_stride + g0 * 8, kn * 16, &full[st]);
-      if (vn)
-        bulk_g2s(dst + kn * 16, P.v + t * P.row_stride + (vg0 - half) * 8, vn * 16, &full[st]);
-      dst += row_bytes;
+    unsigned char* sdst = ring + static_cast<size_t>(st) * R * row_bytes;
+    const uint16_t* ksrc = P.k + static_cast<int64_t>(r0) * P.row_stride + g0 * 8;
+    const uint16_t* vsrc = P.v + static_cast<int64_t>(r0) * P.row_stride + (vg0 - half) * 8;
+    if constexpr (kBlock) {
+      unsigned char* vdst = sdst + R * kn * 16;
+      if (kn) {
+        if (k_packed) {
+          bulk_g2s(sdst, ksrc, rows * kn * 16, &full[st]);
+        } else {
+          for (int r = 0; r < rows; ++r)
+            bulk_g2s(sdst + r * kn * 16, ksrc + static_cast<int64_t>(r) * P.row_stride, kn * 16,
+                     &full[st]);
+        }
+      }
+      if (vn) {
+        if (v_packed) {
+          bulk_g2s(vdst, vsrc, rows * vn * 16, &full[st]);
+        } else {
+          for (int r = 0; r < rows; ++r)
+            bulk_g2s(vdst + r * vn * 16, vsrc + static_cast<int64_t>(r) * P.row_stride, vn * 16,
+                     &full[st]);
+        }
+      }
+    } else {
+      for (int r = 0; r < rows; ++r) {
+        const int64_t o = static_cast<int64_t>(r) * P.row_stride;
+        if (kn) bulk_g2s(sdst, ksrc + o, kn * 16, &full[st]);
+        if (vn) bulk_g2s(sdst + kn * 16, vsrc + o, vn * 16, &full[st]);
+        sdst += row_bytes;
+      }
     }
   };
   int issued = 0;  // chunks issued so far (thread 0 only)
@@ -418,7 +472,11 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }                                                                               \
   } while (0)
   // inactive lanes read column 0 (and never store): no predicated loads
-  const unsigned char* my_ring = ring + (active ? lg : 0) * 16;
+  const unsigned char* my_ring =
+      !kBlock ? ring + (active ? lg : 0) * 16
+              : ring + (!active ? 0 : lg < kn ? lg * 16 : R * kn * 16 + (lg - kn) * 16);
+  // bytes between consecutive rows of this thread's part of a stage
+  const int my_rs = !kBlock ? row_bytes : (active && lg >= kn) ? vn * 16 : kn * 16;
   // slot_mapping is read one 32-row window ahead of use, lane l holding row
   // (window start + l), so its load latency hides behind four chunks.
   constexpr int SW = (32 / R) * R;
@@ -457,7 +515,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       uint4 xr[R];
 #pragma unroll
       for (int r = 0; r < R; ++r)
-        xr[r] = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+        xr[r] = *reinterpret_cast<const uint4*>(stage + r * my_rs);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       released = true;
@@ -471,7 +529,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
 #else
 #pragma unroll fast_unroll<W, MX>()
       for (int r = 0; r < R; ++r) {
-        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
         float2 acc[4];
         conv_step<W>(tw, win, xr, acc);
         const long long off = warp_off[sbase + r];
@@ -487,7 +545,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
           next = (seq + 1 <= S) ? cu(seq + 1) : T;
           start_sequence(seq);
         }
-        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * row_bytes);
+        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
         float2 acc[4];
         conv_step<W>(tw, win, xr, acc);
         const long long off = warp_off[sbase + r];

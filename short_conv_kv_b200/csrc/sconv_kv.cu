@@ -260,6 +260,8 @@ int prefill_impl(
   if (ctas > by_tokens) ctas = by_tokens;
   if (ctas < 1) ctas = 1;
   G.ctas = static_cast<int>(ctas);
+  G.cut_q = static_cast<int>(num_tokens / ctas);
+  G.cut_r = static_cast<int>(num_tokens % ctas);
   const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 16 +
                       (G.cu_smem ? 4 * static_cast<size_t>(num_seqs + 1) : 0);
   if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
