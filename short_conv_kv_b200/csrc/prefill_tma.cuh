@@ -8,7 +8,9 @@
 // to the sequence's end), so the CTA holding position 0 of a sequence also
 // holds every position whose window reaches into the old conv_state: that
 // CTA is the only reader of the old state and the only writer of the new
-// one, and no inter-CTA synchronisation is needed.
+// one, and no inter-CTA synchronisation is needed.  A cut moves forward by
+// at most W-2 rows, so each CTA requests the full chunks of its unmoved
+// range before it has read cu_seqlens.
 //
 // Pipeline.  The rows of the CTA's range (the W-1 rows in front of a range
 // that starts inside a sequence are read directly) stream through a ring of
@@ -48,9 +50,6 @@ namespace sconv {
 #ifndef SCONV_PREFILL_SMALL_W_PER_SM
 #define SCONV_PREFILL_SMALL_W_PER_SM 2  // CTAs per SM for W <= 4
 #endif
-#ifndef SCONV_PREFILL_EARLY_RELEASE
-#define SCONV_PREFILL_EARLY_RELEASE 0  // copy a stage to registers, then release it
-#endif
 #ifndef SCONV_PREFILL_BF16_UNROLL
 #define SCONV_PREFILL_BF16_UNROLL 4  // fast-path unroll of the bf16 store for W <= 4
 #endif
@@ -62,9 +61,6 @@ namespace sconv {
 // packed), 0 = row by row (one copy per row part), 2 = per instance as
 // block_layout<W, MX>() says.
 #define SCONV_PREFILL_BLOCK_LAYOUT 2
-#endif
-#ifndef SCONV_PREFILL_LAST_WARP_REFILL
-#define SCONV_PREFILL_LAST_WARP_REFILL 0  // the last warp to release a stage refills it
 #endif
 
 constexpr int kTmaMaxGroups = 256;   // channel groups per CTA slice
@@ -200,10 +196,9 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Gm.smem_ring);
   uint64_t* empty = full + NS;
   volatile int* abort = reinterpret_cast<volatile int*>(empty + NS);
-  int* s_cu = const_cast<int*>(reinterpret_cast<volatile int*>(empty + NS) + 4);
-#if SCONV_PREFILL_LAST_WARP_REFILL
-  int* rel_cnt = reinterpret_cast<int*>(smem + Gm.smem_ring - kTmaOffTableBytes - 64);
-#endif
+  // after the barriers: abort flag (16 bytes), one int per warp (32 bytes),
+  // then cu_seqlens when staged in shared memory
+  int* s_cu = const_cast<int*>(reinterpret_cast<volatile int*>(empty + NS) + 12);
   // per-warp table of the cache row offsets of the current 32-row window
   // (host reserves 8 warps x 32 x 8 bytes right below the barriers)
   long long* warp_off =
@@ -212,67 +207,18 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], ncw);
-#if SCONV_PREFILL_LAST_WARP_REFILL
-      rel_cnt[s] = 0;
-#endif
-    }
-    *abort = 0;
-    mbar_init_fence();
-  }
-  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
-  if (Gm.cu_smem)
-    for (int i = threadIdx.x; i <= S; i += blockDim.x) s_cu[i] = P.cu_seqlens[i];
-  __syncthreads();
-
-  auto cu = [&](int i) -> int { return Gm.cu_smem ? s_cu[i] : __ldg(P.cu_seqlens + i); };
-  // largest i in [0, S-1] with cu[i] <= t
-  auto seq_of = [&](int t) -> int {
-    int lo = 0, hi = S - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cu(mid) <= t) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-  };
-  // start of range b: even cut, moved off positions 1..W-2 of a sequence
-  auto cut = [&](int b) -> int {
-    int s = b * Gm.cut_q + min(b, Gm.cut_r);
-    if (s >= T) return T;
-    if (W > 1) {
-      const int i = seq_of(s);
-      const int a = cu(i), e = cu(i + 1);
-      const int p = s - a;
-      if (p > 0 && p < W - 1) s = a + min(W - 1, e - a);
-      s = min(max(s, 0), T);
-    }
-    return s;
-  };
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    // cu_seqlens must start at 0, end at T and never decrease (the block's
-    // threads check the entries in parallel)
-    bool ok = threadIdx.x != 0 || (cu(0) == 0 && cu(S) == T);
-    for (int i = threadIdx.x; i < S && ok; i += blockDim.x) ok = cu(i) <= cu(i + 1);
-    if (!ok) raise_flag(P.err, kFlagCuSeqlens);
-  }
-  const int ta = cut(blockIdx.x);
-  const int tb = max(ta, cut(blockIdx.x + 1));
-  if (ta >= tb) return;
-  const int seq0 = seq_of(ta);
-  // a range that starts inside a sequence needs the W-1 rows in front of it
-  // (its halo); they are read directly below, so the ring holds exactly the
-  // range's own rows and every full chunk can take the fast path
-  const bool mid_sequence = (W > 1 && ta > cu(seq0));
-  const int first_row = ta;
-  const int nrows = tb - first_row;
-  const int nchunks = (nrows + R - 1) / R;
+  // Even split of the token axis: range b starts at cut_even(b).  The final
+  // cut (below, once cu_seqlens is read) only moves a start forward, by at
+  // most W-2 rows, so the chunks of [cut_even(b), cut_even(b+1)) can be
+  // requested before cu_seqlens arrives.  Chunk c covers rows
+  // first_row + c*R ... whatever the final start is; rows in front of the
+  // final start are skipped by the consumers.
+  auto cut_even = [&](int b) -> int { return min(b * Gm.cut_q + min(b, Gm.cut_r), T); };
+  const int first_row = cut_even(blockIdx.x);
+  int tb = cut_even(blockIdx.x + 1);  // end of the range (final value set below)
 
   // =================================================================== producer
-  // Issue chunk c (rows first_row + c*R ...) into stage `st` (= c % NS,
-  // tracked by the caller without a division).
+  // Issue chunk c into stage `st` (= c % NS, tracked by the caller).
   // Block layout: a stage holds its R rows' K parts (kn*16 bytes each) back
   // to back, then their V parts.  When a part is a whole row of a packed
   // tensor (row_stride == C), the chunk's rows of that part are one
@@ -318,6 +264,84 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
   };
   int issued = 0;  // chunks issued so far (thread 0 only)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncw);
+    }
+    *abort = 0;
+    mbar_init_fence();
+  }
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  if (kBlock && threadIdx.x == 0) {
+    // full chunks that lie inside the even range: requested at once (block
+    // layout only; in the W=4 bf16 instance the extra live values spill at
+    // its 128-register cap, so it requests after the cut)
+    const int spec = min(NS, (tb - first_row) / R);
+    for (; issued < spec; ++issued) issue(issued, issued);
+  }
+  if (Gm.cu_smem)
+    for (int i = threadIdx.x; i <= S; i += blockDim.x) s_cu[i] = P.cu_seqlens[i];
+  __syncthreads();
+
+  auto cu = [&](int i) -> int { return Gm.cu_smem ? s_cu[i] : __ldg(P.cu_seqlens + i); };
+  // largest i in [0, S-1] with cu[i] <= t
+  auto seq_of = [&](int t) -> int {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu(mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  // start of range b: even cut, moved off positions 1..W-2 of a sequence
+  static_assert(R > W - 2, "a moved cut must stay inside the first chunk");
+  auto cut = [&](int b) -> int {
+    const int s0 = cut_even(b);
+    if (s0 >= T) return T;
+    int s = s0;
+    if (W > 1) {
+      const int i = seq_of(s);
+      const int a = cu(i), e = cu(i + 1);
+      const int p = s - a;
+      if (p > 0 && p < W - 1) s = a + min(W - 1, e - a);
+      // never backwards nor by W-1 or more rows, even for a malformed
+      // cu_seqlens (which is flagged below)
+      s = min(max(s, s0), min(s0 + W - 2, T));
+    }
+    return s;
+  };
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    // cu_seqlens must start at 0, end at T and never decrease (the block's
+    // threads check the entries in parallel)
+    bool ok = threadIdx.x != 0 || (cu(0) == 0 && cu(S) == T);
+    for (int i = threadIdx.x; i < S && ok; i += blockDim.x) ok = cu(i) <= cu(i + 1);
+    if (!ok) raise_flag(P.err, kFlagCuSeqlens);
+  }
+  const int ta = cut(blockIdx.x);
+  // rows of chunk 0 in front of ta, one copy per warp in shared memory (read
+  // once per 32-row window: a register here spills in the W=4 bf16 instance)
+  volatile int* s_skip = abort + 4 + warp;
+  if (lane == 0) *s_skip = ta - first_row;
+  __syncwarp();
+  tb = max(ta, cut(blockIdx.x + 1));
+  if (ta >= tb) return;
+  // The CTA walks rows from first_row.  Rows first_row .. ta-1 (at most W-2,
+  // all in chunk 0) belong to the previous range: they only fill the
+  // window, and their stores are masked through the slot table.  A moved
+  // cut puts ta at position W-1 of its sequence (the window then holds
+  // rows 0 .. W-2 of it) or at a sequence start (whose window is loaded
+  // from its state).  An empty range has requested nothing: its even range
+  // is shorter than W-1 < R rows.
+  const int seq0 = seq_of(first_row);
+  // a walk that starts inside a sequence needs the W-1 rows in front of
+  // first_row (its halo); they are read directly below, so the ring holds
+  // exactly the walked rows and every full chunk can take the fast path
+  const bool mid_sequence = (W > 1 && first_row > cu(seq0));
+  const int nrows = tb - first_row;
+  const int nchunks = (nrows + R - 1) / R;
+
   // After giving up, let the copies already issued land before the CTA's
   // shared memory can be released (bounded as well).
   auto drain = [&]() {
@@ -447,11 +471,12 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     int64_t si;
     skip = !check_sequence(seq, si);
     if constexpr (W > 1) {
-      // halo: rows ta-(W-1) .. ta-1 of the same sequence (the cut rule puts
-      // ta at position >= W-1, so they are never state rows)
+      // halo: rows first_row-(W-1) .. first_row-1.  When first_row == ta
+      // (the cut did not move) they lie in ta's sequence at positions >= 0,
+      // never in the state; otherwise they only feed the masked rows.
 #pragma unroll
       for (int j = 0; j < W - 1; ++j) {
-        const int64_t q = static_cast<int64_t>(ta) - (W - 1) + j;
+        const int64_t q = static_cast<int64_t>(first_row) - (W - 1) + j;
         const uint4 h = (active && q >= 0) ? ld_ro(xbase + q * P.row_stride) : make_uint4(0, 0, 0, 0);
         unpack8(h, win[j]);
       }
@@ -500,33 +525,17 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     const int rows = min(R, tb - r0);
     if (c % (SW / R) == 0) {
       // rows [r0, r0 + SW): lane l writes row r0 + l's cache row offset
+      // (-1, masked, for the rows of chunk 0 in front of ta)
       __syncwarp();
-      warp_off[lane] = slot_row_offset(P, next_slot, report_slots);
+      warp_off[lane] = (c == 0 && lane < *s_skip) ? -1 : slot_row_offset(P, next_slot, report_slots);
       __syncwarp();
       next_slot = load_slot(c / (SW / R) + 1);
     }
     const int sbase = (c % (SW / R)) * R;  // this chunk's first lane
     const unsigned char* stage = my_ring + static_cast<size_t>(s) * R * row_bytes;
-    bool released = false;
     if (next >= r0 + rows && !skip) {
       // fast path: up to R tokens of one sequence, no branches (rows past
       // the end of the range compute on stale data and are not stored)
-#if SCONV_PREFILL_EARLY_RELEASE
-      uint4 xr[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        xr[r] = *reinterpret_cast<const uint4*>(stage + r * my_rs);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      released = true;
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float2 acc[4];
-        conv_step<W>(tw, win, xr[r], acc);
-        const long long off = warp_off[sbase + r];
-        NORM_STORE(active && r < rows && off >= 0);
-      }
-#else
 #pragma unroll fast_unroll<W, MX>()
       for (int r = 0; r < R; ++r) {
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
@@ -535,7 +544,6 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
         const long long off = warp_off[sbase + r];
         NORM_STORE(active && r < rows && off >= 0);
       }
-#endif
     } else {
       for (int r = 0; r < rows; ++r) {
         const int t = r0 + r;
@@ -553,25 +561,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       }
     }
     __syncwarp();
-#if SCONV_PREFILL_LAST_WARP_REFILL
-    if (lane == 0) {
-      __threadfence_block();
-      if (atomicAdd(&rel_cnt[s], 1) == ncw - 1) {
-        rel_cnt[s] = 0;
-        if (c + NS < nchunks) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(c + NS, s);
-        }
-      }
-    }
-    (void)released;
-    if (++s == NS) {
-      s = 0;
-      ph ^= 1;
-    }
-    continue;
-#endif
-    if (lane == 0 && !released) mbar_arrive(&empty[s]);  // stage fully consumed
+    if (lane == 0) mbar_arrive(&empty[s]);  // stage fully consumed
     if (threadIdx.x == 0 && c >= 1 && issued < nchunks) {
       // refill the stage of chunk c-1 (issued == c-1+NS lands there) once
       // every warp has released it

@@ -249,9 +249,6 @@ int prefill_impl(
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
   // + per-warp slot-offset tables + per-thread gammas
   G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes + sconv::kTmaGammaBytes;
-#if SCONV_PREFILL_LAST_WARP_REFILL
-  G.smem_ring += 64;  // release counters
-#endif
   G.cu_smem = num_seqs < sconv::kTmaCuSmemMax ? 1 : 0;
   G.timeout_ns = 1000000000ull;
   const int64_t resident = static_cast<int64_t>(sm_count()) * per_sm;
@@ -262,7 +259,7 @@ int prefill_impl(
   G.ctas = static_cast<int>(ctas);
   G.cut_q = static_cast<int>(num_tokens / ctas);
   G.cut_r = static_cast<int>(num_tokens % ctas);
-  const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 16 +
+  const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 48 +
                       (G.cu_smem ? 4 * static_cast<size_t>(num_seqs + 1) : 0);
   if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
     snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
