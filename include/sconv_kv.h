@@ -225,6 +225,64 @@ SCONV_KV_API int sconv_kv_decode_mxfp8(
     uint8_t* v_scale, const sconv_kv_cache_layout_t* layout, int* err_flag,
     void* stream);
 
+/*
+ * Unfused stages.  The same step as four separate passes over HBM, each
+ * with its intermediate in bf16: the chain that the fused entry points
+ * replace ("SGLang and Miles announce day-0 Inkling support", aib.vote
+ * English news item, paragraph 2: K/V conv, normalisation and KV-cache
+ * write fused, against an unfused chain).  Run in order on one stream:
+ *
+ *   sconv_kv_stage_conv          k, v, old state  -> y
+ *   sconv_kv_stage_rmsnorm       y                -> z
+ *   sconv_kv_stage_scatter       z, slot_mapping  -> k_cache, v_cache
+ *   sconv_kv_stage_state_update  k, v, old state  -> new state
+ *
+ * the result equals the fused step's except that y is rounded to bf16
+ * before the normalisation.  Each stage is also usable alone.
+ *
+ * Intermediates y and z: bf16 [num_tokens, 2*num_kv_heads*head_dim]
+ * (K channels, then V), device memory owned by the caller, 16-byte
+ * aligned.  Other arguments mean what they mean for
+ * sconv_kv_prefill_varlen, with the same layouts, alignment rules and
+ * flag bits.  Calls with num_tokens == 0 (or num_seqs == 0) enqueue nothing
+ * and succeed without looking at the pointers.
+ *
+ * sconv_kv_stage_conv: y[t] = sum_j w[j] * x[t-W+1+j] per channel, rows
+ *   before a sequence's first token taken from its conv_state (read only).
+ *   A bad state index or a malformed cu_seqlens skips the token (y not
+ *   written) and sets the flag bit.
+ * sconv_kv_stage_rmsnorm: z = y / sqrt(mean over the head of y^2 + eps) *
+ *   gamma[d] per (token, head), rounded to bf16.
+ * sconv_kv_stage_scatter: cache[slot_mapping[t]] = z[t] (K half into
+ *   k_cache, V half into v_cache); slot < 0 skips the token; a slot past
+ *   the cache is skipped and flagged.
+ * sconv_kv_stage_state_update: each sequence's state = the last W-1 raw
+ *   rows of (old state ++ its rows), in place; must run after every reader
+ *   of the old state (sconv_kv_stage_conv).  W == 1 has no state: no-op.
+ */
+SCONV_KV_API int sconv_kv_stage_conv(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, int W, int num_kv_heads, int head_dim,
+    const void* conv_state, const int32_t* state_indices,
+    int64_t state_pool_size, void* y, int* err_flag, void* stream);
+
+SCONV_KV_API int sconv_kv_stage_rmsnorm(
+    const void* y, int64_t num_tokens, const float* gamma_k,
+    const float* gamma_v, float eps, int num_kv_heads, int head_dim, void* z,
+    void* stream);
+
+SCONV_KV_API int sconv_kv_stage_scatter(
+    const void* z, int64_t num_tokens, int num_kv_heads, int head_dim,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
+
+SCONV_KV_API int sconv_kv_stage_state_update(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, int W, int num_kv_heads,
+    int head_dim, void* conv_state, const int32_t* state_indices,
+    int64_t state_pool_size, int* err_flag, void* stream);
+
 /* Static text for a status code (never NULL). */
 SCONV_KV_API const char* sconv_kv_strerror(int status);
 

@@ -65,6 +65,16 @@ def _load(path):
         vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
         vp, vp, vp, vp, lp, ip, vp]
     lib.sconv_kv_decode_mxfp8.restype = i32
+    lib.sconv_kv_stage_conv.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp, i64, vp, ip, vp]
+    lib.sconv_kv_stage_conv.restype = i32
+    lib.sconv_kv_stage_rmsnorm.argtypes = [vp, i64, vp, vp, f32, i32, i32, vp, vp]
+    lib.sconv_kv_stage_rmsnorm.restype = i32
+    lib.sconv_kv_stage_scatter.argtypes = [vp, i64, i32, i32, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_stage_scatter.restype = i32
+    lib.sconv_kv_stage_state_update.argtypes = [
+        vp, vp, i64, i64, vp, i32, i32, i32, i32, vp, vp, i64, ip, vp]
+    lib.sconv_kv_stage_state_update.restype = i32
     lib.sconv_kv_strerror.argtypes = [i32]
     lib.sconv_kv_strerror.restype = ctypes.c_char_p
     lib.sconv_kv_last_cuda_error.argtypes = []
@@ -342,3 +352,93 @@ def prepare_decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_s
             _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale),
             ctypes.byref(lay), _ptr(err_flag), _stream(stream))
     return PreparedCall("sconv_kv_decode_mxfp8", args, keep_alive=(lay,))
+
+
+# ---------------------------------------------------------------- unfused stages
+
+def _check(rc, name):
+    if rc != OK:
+        raise SconvKVError(rc, name)
+
+
+def stage_conv(k, v, cu_seqlens, conv_w_k, conv_w_v, conv_state, y, state_indices=None,
+               err_flag=None, stream=None):
+    """Pass 1 of the unfused chain: y (bf16 [T, 2*Hkv*D], K then V) = the
+    causal conv of k and v; conv_state is only read."""
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    W = conv_w_k.shape[0]
+    H, D = (k.shape[1], k.shape[2]) if k.dim() == 3 else (None, None)
+    if H is None:
+        raise ValueError("k must be [T, Hkv, D] for the stage entry points")
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    _check(_lib.sconv_kv_stage_conv(
+        kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1, _ptr(conv_w_k),
+        _ptr(conv_w_v), W, H, D, _ptr(conv_state) if W > 1 else None, _ptr(state_indices),
+        pool, _ptr(y), _ptr(err_flag), _stream(stream)), "sconv_kv_stage_conv")
+
+
+def stage_rmsnorm(y, gamma_k, gamma_v, eps, num_kv_heads, z, stream=None):
+    """Pass 2: z = per-head RMSNorm of y times gamma (bf16 [T, 2*Hkv*D])."""
+    D = gamma_k.shape[0]
+    _check(_lib.sconv_kv_stage_rmsnorm(_ptr(y), y.shape[0], _ptr(gamma_k), _ptr(gamma_v),
+                                       float(eps), int(num_kv_heads), D, _ptr(z),
+                                       _stream(stream)), "sconv_kv_stage_rmsnorm")
+
+
+def stage_scatter(z, slot_mapping, k_cache, v_cache, err_flag=None, stream=None):
+    """Pass 3: cache[slot_mapping[t]] = z[t] (K half / V half)."""
+    lay = layout_of(k_cache)
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    _check(_lib.sconv_kv_stage_scatter(_ptr(z), z.shape[0], H, D, _ptr(slot_mapping),
+                                       _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
+                                       _ptr(err_flag), _stream(stream)), "sconv_kv_stage_scatter")
+
+
+def stage_state_update(k, v, cu_seqlens, W, conv_state, state_indices=None, err_flag=None,
+                       stream=None):
+    """Pass 4: conv_state <- last W-1 raw rows of (old state ++ rows), in place."""
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    H, D = k.shape[1], k.shape[2]
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    _check(_lib.sconv_kv_stage_state_update(
+        kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1, int(W), H, D,
+        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(err_flag),
+        _stream(stream)), "sconv_kv_stage_state_update")
+
+
+def prepare_unfused(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
+                    slot_mapping, k_cache, v_cache, y, z, state_indices=None, err_flag=None,
+                    stream=None):
+    """The four stage calls of one step, pre-marshalled (conv, rmsnorm,
+    scatter, state update, in that order on one stream)."""
+    kp, rs = _rows(k, "k")
+    vp, _ = _rows(v, "v")
+    W = conv_w_k.shape[0]
+    T, H, D = k.shape[0], k.shape[1], k.shape[2]
+    S = cu_seqlens.shape[0] - 1
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    st = _ptr(conv_state) if W > 1 else None
+    lay = layout_of(k_cache)
+    sp = _stream(stream)
+    calls = [
+        PreparedCall("sconv_kv_stage_conv", (kp, vp, rs, T, _ptr(cu_seqlens), S, _ptr(conv_w_k),
+                                             _ptr(conv_w_v), W, H, D, st, _ptr(state_indices),
+                                             pool, _ptr(y), _ptr(err_flag), sp)),
+        PreparedCall("sconv_kv_stage_rmsnorm", (_ptr(y), T, _ptr(gamma_k), _ptr(gamma_v),
+                                                ctypes.c_float(eps), H, D, _ptr(z), sp)),
+        PreparedCall("sconv_kv_stage_scatter", (_ptr(z), T, H, D, _ptr(slot_mapping),
+                                                _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
+                                                _ptr(err_flag), sp), keep_alive=(lay,)),
+        PreparedCall("sconv_kv_stage_state_update", (kp, vp, rs, T, _ptr(cu_seqlens), S, W, H, D,
+                                                     st, _ptr(state_indices), pool,
+                                                     _ptr(err_flag), sp)),
+    ]
+
+    def run():
+        for c in calls:
+            c()
+    return run

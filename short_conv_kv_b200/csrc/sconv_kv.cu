@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "decode_tma.cuh"
 #include "prefill_tma.cuh"
+#include "stages.cuh"
 
 namespace {
 
@@ -325,6 +326,73 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
                 stream);
 }
 
+// ---- unfused stages
+
+using StageFn = void (*)(sconv::StageParams);
+
+template <int W>
+StageFn stage_conv_fn() { return sconv::stage_conv_kernel<W>; }
+template <int W>
+StageFn stage_state_fn() { return sconv::stage_state_kernel<W>; }
+
+StageFn stage_conv_by_w(int W) {
+  switch (W) {
+    case 1: return stage_conv_fn<1>();
+    case 2: return stage_conv_fn<2>();
+    case 3: return stage_conv_fn<3>();
+    case 4: return stage_conv_fn<4>();
+    case 5: return stage_conv_fn<5>();
+    case 6: return stage_conv_fn<6>();
+    case 7: return stage_conv_fn<7>();
+    case 8: return stage_conv_fn<8>();
+    default: return nullptr;
+  }
+}
+StageFn stage_state_by_w(int W) {
+  switch (W) {
+    case 2: return stage_state_fn<2>();
+    case 3: return stage_state_fn<3>();
+    case 4: return stage_state_fn<4>();
+    case 5: return stage_state_fn<5>();
+    case 6: return stage_state_fn<6>();
+    case 7: return stage_state_fn<7>();
+    case 8: return stage_state_fn<8>();
+    default: return nullptr;
+  }
+}
+StageFn stage_rmsnorm_by_d(int D) {
+  switch (D) {
+    case 64: return sconv::stage_rmsnorm_kernel<64>;
+    case 128: return sconv::stage_rmsnorm_kernel<128>;
+    case 256: return sconv::stage_rmsnorm_kernel<256>;
+    default: return nullptr;
+  }
+}
+
+// Shape checks shared by the stages; fills the channel counts of P.
+int stage_shape(int num_kv_heads, int head_dim, int64_t num_tokens, sconv::StageParams* P) {
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return SCONV_KV_ERR_SHAPE;
+  if (num_kv_heads < 1 || num_kv_heads > (1 << 16)) return SCONV_KV_ERR_SHAPE;
+  if (num_tokens < 0 || num_tokens > INT32_MAX) return SCONV_KV_ERR_SHAPE;
+  memset(P, 0, sizeof(*P));
+  P->C = num_kv_heads * head_dim;
+  P->D = head_dim;
+  P->NG = 2 * P->C / 8;
+  P->num_tokens = num_tokens;
+  P->inv_d = 1.0f / static_cast<float>(head_dim);
+  return SCONV_KV_OK;
+}
+
+// Grid-stride launch over `work` items of one thread each.
+int stage_launch(StageFn fn, int64_t work, sconv::StageParams* P, void* stream) {
+  if (work <= 0) return SCONV_KV_OK;
+  const int64_t want = (work + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  void* args[] = {P};
+  return launch(reinterpret_cast<const void*>(fn), dim3(static_cast<unsigned>(want < cap ? want : cap)),
+                dim3(256), args, 0, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -413,6 +481,111 @@ int sconv_kv_decode_mxfp8(const void* k, const void* v, int64_t row_stride, int 
                      num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
                      slot_mapping, k_data, v_data, layout, err_flag, stream, true, k_scale,
                      v_scale);
+}
+
+int sconv_kv_stage_conv(const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+                        const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+                        const void* conv_w_v, int W, int num_kv_heads, int head_dim,
+                        const void* conv_state, const int32_t* state_indices,
+                        int64_t state_pool_size, void* y, int* err_flag, void* stream) {
+  sconv::StageParams P;
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
+  if (st) return st;
+  if (num_tokens == 0 || num_seqs == 0) return SCONV_KV_OK;
+  if (!k || !v || !cu_seqlens || !conv_w_k || !conv_w_v || !y || (W > 1 && !conv_state))
+    return SCONV_KV_ERR_NULL;
+  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P.C)
+    return SCONV_KV_ERR_SHAPE;
+  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_w_k) ||
+      !aligned16(conv_w_v) || !aligned16(y) || (conv_state && !aligned16(conv_state)))
+    return SCONV_KV_ERR_ALIGN;
+  P.k = static_cast<const uint16_t*>(k);
+  P.v = static_cast<const uint16_t*>(v);
+  P.row_stride = row_stride;
+  P.cu_seqlens = cu_seqlens;
+  P.num_seqs = num_seqs;
+  P.w_k = static_cast<const uint16_t*>(conv_w_k);
+  P.w_v = static_cast<const uint16_t*>(conv_w_v);
+  P.W = W;
+  P.state = const_cast<uint16_t*>(static_cast<const uint16_t*>(conv_state));
+  P.state_indices = state_indices;
+  P.pool = state_pool_size;
+  P.y = static_cast<uint16_t*>(y);
+  P.err = err_flag;
+  return stage_launch(stage_conv_by_w(W), num_tokens * P.NG, &P, stream);
+}
+
+int sconv_kv_stage_rmsnorm(const void* y, int64_t num_tokens, const float* gamma_k,
+                           const float* gamma_v, float eps, int num_kv_heads, int head_dim,
+                           void* z, void* stream) {
+  sconv::StageParams P;
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
+  if (st) return st;
+  if (num_tokens == 0) return SCONV_KV_OK;
+  if (!y || !gamma_k || !gamma_v || !z) return SCONV_KV_ERR_NULL;
+  if (!aligned16(y) || !aligned16(z) || !aligned16(gamma_k) || !aligned16(gamma_v))
+    return SCONV_KV_ERR_ALIGN;
+  P.y = const_cast<uint16_t*>(static_cast<const uint16_t*>(y));
+  P.z = static_cast<uint16_t*>(z);
+  P.gamma_k = gamma_k;
+  P.gamma_v = gamma_v;
+  P.eps = eps;
+  return stage_launch(stage_rmsnorm_by_d(head_dim), num_tokens * P.NG, &P, stream);
+}
+
+int sconv_kv_stage_scatter(const void* z, int64_t num_tokens, int num_kv_heads, int head_dim,
+                           const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                           const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  sconv::StageParams P;
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
+  if (st) return st;
+  if (num_tokens == 0) return SCONV_KV_OK;
+  if (!z || !slot_mapping || !k_cache || !v_cache || !layout) return SCONV_KV_ERR_NULL;
+  if (layout->num_kv_heads != num_kv_heads || layout->head_dim != head_dim ||
+      layout->num_pages < 0 || layout->page_size < 1 || layout->stride_head < head_dim ||
+      layout->stride_slot < 1 || layout->stride_page < 1)
+    return SCONV_KV_ERR_SHAPE;
+  if (!aligned16(z) || !aligned16(k_cache) || !aligned16(v_cache) || layout->stride_head % 8 ||
+      layout->stride_slot % 8 || layout->stride_page % 8)
+    return SCONV_KV_ERR_ALIGN;
+  P.z = const_cast<uint16_t*>(static_cast<const uint16_t*>(z));
+  P.slots = slot_mapping;
+  P.k_cache = static_cast<uint16_t*>(k_cache);
+  P.v_cache = static_cast<uint16_t*>(v_cache);
+  P.num_slots = layout->num_pages * layout->page_size;
+  P.page_size = layout->page_size;
+  P.stride_page = layout->stride_page;
+  P.stride_slot = layout->stride_slot;
+  P.stride_head = layout->stride_head;
+  P.err = err_flag;
+  return stage_launch(sconv::stage_scatter_kernel, num_tokens * P.NG, &P, stream);
+}
+
+int sconv_kv_stage_state_update(const void* k, const void* v, int64_t row_stride,
+                                int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
+                                int W, int num_kv_heads, int head_dim, void* conv_state,
+                                const int32_t* state_indices, int64_t state_pool_size,
+                                int* err_flag, void* stream) {
+  sconv::StageParams P;
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
+  if (st) return st;
+  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P.C)
+    return SCONV_KV_ERR_SHAPE;
+  if (W == 1 || num_seqs == 0) return SCONV_KV_OK;  // no state rows
+  if (!k || !v || !cu_seqlens || !conv_state) return SCONV_KV_ERR_NULL;
+  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_state))
+    return SCONV_KV_ERR_ALIGN;
+  P.k = static_cast<const uint16_t*>(k);
+  P.v = static_cast<const uint16_t*>(v);
+  P.row_stride = row_stride;
+  P.cu_seqlens = cu_seqlens;
+  P.num_seqs = num_seqs;
+  P.W = W;
+  P.state = static_cast<uint16_t*>(conv_state);
+  P.state_indices = state_indices;
+  P.pool = state_pool_size;
+  P.err = err_flag;
+  return stage_launch(stage_state_by_w(W), static_cast<int64_t>(num_seqs) * P.NG, &P, stream);
 }
 
 }  // extern "C"
