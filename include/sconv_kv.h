@@ -67,6 +67,7 @@ extern "C" {
 #define SCONV_KV_ERR_ALIGN (-3)       /* pointer or stride not 16-byte aligned */
 #define SCONV_KV_ERR_UNSUPPORTED (-4) /* valid but not implemented combination */
 #define SCONV_KV_ERR_CUDA (-5)        /* CUDA reported an error at launch     */
+#define SCONV_KV_ERR_SCRATCH (-6)     /* call needs more than the static scratch */
 
 /* ---------------------------------------------------- device-side flag bits */
 #define SCONV_KV_FLAG_SLOT_RANGE 1   /* slot >= num_pages*page_size: skipped  */
@@ -282,6 +283,35 @@ SCONV_KV_API int sconv_kv_stage_state_update(
     const int32_t* cu_seqlens, int num_seqs, int W, int num_kv_heads,
     int head_dim, void* conv_state, const int32_t* state_indices,
     int64_t state_pool_size, int* err_flag, void* stream);
+
+/*
+ * The unfused chain in one call, with no allocation: the same four stages
+ * (conv, rmsnorm, scatter, state update, in that order on `stream`), their
+ * bf16 intermediates y and z placed in a scratch buffer that the library
+ * holds in static device memory (SCONV_KV_NOALLOC_SCRATCH_BYTES per device,
+ * reserved when the library's module loads; its address is looked up once
+ * per device).  The library allocates nothing on any call.
+ *
+ * Arguments and results as for sconv_kv_prefill_varlen (bf16 caches), and
+ * the results equal those of the four sconv_kv_stage_* calls.  The call
+ * needs 2 * round_up_256(num_tokens * 2 * num_kv_heads * head_dim * 2)
+ * bytes of scratch; a larger call returns SCONV_KV_ERR_SCRATCH before
+ * enqueueing anything.  Calls share the one scratch buffer: they must be
+ * ordered (one stream, or streams ordered by events).
+ *
+ * The source pages have no counterpart to this entry point: it is a
+ * convenience of this library.
+ */
+#define SCONV_KV_NOALLOC_SCRATCH_BYTES (64ll << 20)
+
+SCONV_KV_API int sconv_kv_unfused_step_noalloc(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
 
 /* Static text for a status code (never NULL). */
 SCONV_KV_API const char* sconv_kv_strerror(int status);

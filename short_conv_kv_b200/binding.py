@@ -18,7 +18,8 @@ LIB_PATH = os.environ.get("SCONV_KV_LIB", _build.LIB)
 
 # status codes and device flag bits (values fixed by include/sconv_kv.h)
 OK = 0
-ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA = -1, -2, -3, -4, -5
+ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_SCRATCH = -1, -2, -3, -4, -5, -6
+NOALLOC_SCRATCH_BYTES = 64 << 20
 FLAG_SLOT_RANGE, FLAG_STATE_INDEX, FLAG_CU_SEQLENS, FLAG_TIMEOUT = 1, 2, 4, 8
 MAX_W = 8
 
@@ -75,6 +76,10 @@ def _load(path):
     lib.sconv_kv_stage_state_update.argtypes = [
         vp, vp, i64, i64, vp, i32, i32, i32, i32, vp, vp, i64, ip, vp]
     lib.sconv_kv_stage_state_update.restype = i32
+    lib.sconv_kv_unfused_step_noalloc.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp,
+        i64, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_unfused_step_noalloc.restype = i32
     lib.sconv_kv_strerror.argtypes = [i32]
     lib.sconv_kv_strerror.restype = ctypes.c_char_p
     lib.sconv_kv_last_cuda_error.argtypes = []
@@ -442,3 +447,26 @@ def prepare_unfused(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
         for c in calls:
             c()
     return run
+
+
+def unfused_step_noalloc(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
+                         conv_state, slot_mapping, k_cache, v_cache, state_indices=None,
+                         err_flag=None, stream=None):
+    """The four unfused stages in one call, intermediates in the library's
+    static scratch (no allocation); same arguments as prefill_varlen.
+    Raises SconvKVError with code ERR_SCRATCH when the batch needs more than
+    NOALLOC_SCRATCH_BYTES of scratch."""
+    kp, rs = _rows(k, "k")
+    vp, rs_v = _rows(v, "v")
+    if rs != rs_v:
+        raise ValueError("k and v must share the row stride")
+    W = conv_w_k.shape[0]
+    H, D = k_cache.shape[2], k_cache.shape[3]
+    lay = layout_of(k_cache)
+    pool = conv_state.shape[0] if conv_state is not None else 0
+    _check(_lib.sconv_kv_unfused_step_noalloc(
+        kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1, _ptr(conv_w_k),
+        _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v), float(eps), W, H, D,
+        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(slot_mapping),
+        _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay), _ptr(err_flag), _stream(stream)),
+        "sconv_kv_unfused_step_noalloc")

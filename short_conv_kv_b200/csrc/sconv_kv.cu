@@ -393,6 +393,27 @@ int stage_launch(StageFn fn, int64_t work, sconv::StageParams* P, void* stream) 
                 dim3(256), args, 0, stream);
 }
 
+// ---- static scratch of the no-alloc unfused step (y, then z)
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[SCONV_KV_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch on the current device, looked up once per
+// device (nullptr if the lookup fails).
+unsigned char* noalloc_scratch() {
+  static unsigned char* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    cached[dev] = static_cast<unsigned char*>(p);
+  }
+  return cached[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -407,6 +428,7 @@ const char* sconv_kv_strerror(int status) {
     case SCONV_KV_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
     case SCONV_KV_ERR_UNSUPPORTED: return "unsupported combination";
     case SCONV_KV_ERR_CUDA: return "CUDA error at launch (see sconv_kv_last_cuda_error)";
+    case SCONV_KV_ERR_SCRATCH: return "call needs more than the static scratch buffer";
     default: return "unknown status";
   }
 }
@@ -481,6 +503,41 @@ int sconv_kv_decode_mxfp8(const void* k, const void* v, int64_t row_stride, int 
                      num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
                      slot_mapping, k_data, v_data, layout, err_flag, stream, true, k_scale,
                      v_scale);
+}
+
+int sconv_kv_unfused_step_noalloc(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+  if (num_tokens < 0 || num_kv_heads < 1 || head_dim < 1) return SCONV_KV_ERR_SHAPE;
+  if (num_tokens == 0 || num_seqs == 0) return SCONV_KV_OK;
+  const int64_t bytes = num_tokens * 2 * static_cast<int64_t>(num_kv_heads) * head_dim * 2;
+  const int64_t part = (bytes + 255) / 256 * 256;
+  if (2 * part > SCONV_KV_NOALLOC_SCRATCH_BYTES) return SCONV_KV_ERR_SCRATCH;
+  unsigned char* scratch = noalloc_scratch();
+  if (!scratch) {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "scratch address lookup failed");
+    return SCONV_KV_ERR_CUDA;
+  }
+  void* y = scratch;
+  void* z = scratch + part;
+  int st = sconv_kv_stage_conv(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k,
+                               conv_w_v, W, num_kv_heads, head_dim, conv_state, state_indices,
+                               state_pool_size, y, err_flag, stream);
+  if (st) return st;
+  st = sconv_kv_stage_rmsnorm(y, num_tokens, gamma_k, gamma_v, eps, num_kv_heads, head_dim, z,
+                              stream);
+  if (st) return st;
+  st = sconv_kv_stage_scatter(z, num_tokens, num_kv_heads, head_dim, slot_mapping, k_cache,
+                              v_cache, layout, err_flag, stream);
+  if (st) return st;
+  return sconv_kv_stage_state_update(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, W,
+                                     num_kv_heads, head_dim, conv_state, state_indices,
+                                     state_pool_size, err_flag, stream);
 }
 
 int sconv_kv_stage_conv(const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
