@@ -95,6 +95,27 @@ def load(path=None):
          ctypes.c_double, _int, _int, _int, _u16p, _i32p, _i64, _i64p,
          _u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64, _i64, _f64p, _f64p])
     lib.oracle_prefill_varlen_mxfp8.restype = _int
+    # layout variants: per-head gamma stride, ring-buffer state positions
+    lib.oracle_rmsnorm_strided.argtypes = [_f64p, _i64, _int, _int, _f32p, _i64,
+                                           ctypes.c_double, _f64p]
+    lib.oracle_rmsnorm_strided.restype = None
+    lib.oracle_state_update_ring.argtypes = [_u16p, _i64, _i64, _u16p, _i64, _int, _int, _i64]
+    lib.oracle_state_update_ring.restype = None
+    lib.oracle_prefill_varlen_opts.argtypes = (
+        [_u16p, _u16p, _i64, _i64, _i32p, _int, _u16p, _u16p, _f32p, _f32p, _i64,
+         ctypes.c_double, _int, _int, _int, _u16p, _i32p, _i64p, _i64, _i64p, _u16p, _u16p,
+         _i64, _i64, _i64, _i64, _i64, _f64p, _f64p])
+    lib.oracle_prefill_varlen_opts.restype = _int
+    lib.oracle_decode_opts.argtypes = (
+        [_u16p, _u16p, _i64, _int, _u16p, _u16p, _f32p, _f32p, _i64, ctypes.c_double, _int,
+         _int, _int, _u16p, _i32p, _i64p, _i64, _i64p, _u16p, _u16p, _i64, _i64, _i64, _i64,
+         _i64, _f64p, _f64p])
+    lib.oracle_decode_opts.restype = _int
+    lib.oracle_prefill_varlen_mxfp8_opts.argtypes = (
+        [_u16p, _u16p, _i64, _i64, _i32p, _int, _u16p, _u16p, _f32p, _f32p, _i64,
+         ctypes.c_double, _int, _int, _int, _u16p, _i32p, _i64p, _i64, _i64p,
+         _u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64, _i64, _f64p, _f64p])
+    lib.oracle_prefill_varlen_mxfp8_opts.restype = _int
     if path == _build.LIB:
         _lib = lib
     return lib
@@ -156,10 +177,10 @@ def rmsnorm(y, num_heads, gamma, eps, lib=None):
     y = np.ascontiguousarray(y, dtype=np.float64)
     gamma = np.ascontiguousarray(gamma, dtype=np.float32)
     L = y.shape[0]
-    D = gamma.shape[0]
+    D = gamma.shape[-1]
     z = np.empty_like(y)
-    lib.oracle_rmsnorm(_p(y, _f64p), L, num_heads, D, _p(gamma, _f32p),
-                       float(eps), _p(z, _f64p))
+    lib.oracle_rmsnorm_strided(_p(y, _f64p), L, num_heads, D, _p(gamma, _f32p),
+                               D if gamma.ndim == 2 else 0, float(eps), _p(z, _f64p))
     return z
 
 
@@ -188,18 +209,51 @@ def state_update(x, state, lib=None):
     return s
 
 
+def _gammas(gamma_k, gamma_v, H):
+    """float32 gammas and their head stride: [D] (shared by every head,
+    stride 0) or [H, D] (one per head, stride D)."""
+    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
+    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    assert gk.shape == gv.shape and gk.ndim in (1, 2)
+    if gk.ndim == 2:
+        assert gk.shape[0] == H
+        return gk, gv, gk.shape[1]
+    return gk, gv, 0
+
+
+def _positions(state_positions):
+    return None if state_positions is None else np.ascontiguousarray(state_positions, np.int64)
+
+
+def state_update_ring(x, state, pos0, lib=None):
+    """Step a5 with a ring-buffer state (position p in row p mod (W-1)) for
+    one tensor of one sequence that has seen pos0 tokens; returns the new
+    state rows."""
+    lib = lib or load()
+    x = _u16(x)
+    s = _u16(state).copy()
+    n, C = s.shape
+    lib.oracle_state_update_ring(_p(x, _u16p), C, x.shape[0], _p(s, _u16p), C, C, n + 1,
+                                 int(pos0))
+    return s
+
+
 # ---------------------------------------------------------------- whole step
 
 def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                    eps, conv_state, slot_mapping, k_cache, v_cache,
-                   state_indices=None, want_z=True, check=True, lib=None):
+                   state_indices=None, want_z=True, check=True, lib=None,
+                   state_positions=None):
     """The whole step (a1..a5) over a varlen batch.
 
     k, v: uint16 [T, H, D] (or [T, C]); cu_seqlens int32 [S+1];
-    conv_w_*: uint16 [W, C]; gamma_*: float32 [D]; conv_state: uint16
-    [pool, W-1, 2C]; slot_mapping int64 [T]; caches uint16
-    [num_pages, page_size, H, D].  Inputs are not modified: returns
-    dict(k_cache, v_cache, conv_state, z_k, z_v, status) with fresh arrays.
+    conv_w_*: uint16 [W, C]; gamma_*: float32 [D] (shared by every head) or
+    [H, D] (per head); conv_state: uint16 [pool, W-1, 2C], oldest row first,
+    or, with state_positions (int64 [S], tokens each sequence has seen), a
+    ring in which position p lives in row p mod (W-1); slot_mapping int64
+    [T]; caches uint16 [num_pages, page_size, H, D].  Inputs are not
+    modified: returns dict(k_cache, v_cache, conv_state, z_k, z_v, status)
+    with fresh arrays.
     """
     lib = lib or load()
     k, v = _u16(k), _u16(v)
@@ -209,8 +263,8 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
     k2, v2 = k.reshape(T, C), v.reshape(T, C)
     wk, wv = _u16(conv_w_k), _u16(conv_w_v)
     W = wk.shape[0]
-    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
-    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    gk, gv, ghs = _gammas(gamma_k, gamma_v, H)
+    pos = _positions(state_positions)
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
     S = cu.shape[0] - 1
     st = _u16(conv_state).copy()
@@ -221,11 +275,11 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
         state_indices, dtype=np.int32)
     zk = np.zeros((T, C), np.float64) if want_z else None
     zv = np.zeros((T, C), np.float64) if want_z else None
-    rc = lib.oracle_prefill_varlen(
+    rc = lib.oracle_prefill_varlen_opts(
         _p(k2, _u16p), _p(v2, _u16p), C, T, _p(cu, _i32p), S,
-        _p(wk, _u16p), _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p),
+        _p(wk, _u16p), _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p), ghs,
         float(eps), W, H, D, _p(st if W > 1 else None, _u16p),
-        _p(si, _i32p), pool, _p(sm, _i64p), _p(kc, _u16p), _p(vc, _u16p),
+        _p(si, _i32p), _p(pos, _i64p), pool, _p(sm, _i64p), _p(kc, _u16p), _p(vc, _u16p),
         num_pages, page_size, page_size * C, C, D, _p(zk, _f64p),
         _p(zv, _f64p))
     if check and rc != 0:
@@ -236,19 +290,19 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
 
 def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
            slot_mapping, k_cache, v_cache, state_indices=None, want_z=True,
-           check=True, lib=None):
+           check=True, lib=None, state_positions=None):
     """One decode step: one new token per sequence (k, v: [B, H, D])."""
     B = np.asarray(k).shape[0]
     cu = np.arange(B + 1, dtype=np.int32)
     return prefill_varlen(k, v, cu, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
                           conv_state, slot_mapping, k_cache, v_cache,
                           state_indices=state_indices, want_z=want_z,
-                          check=check, lib=lib)
+                          check=check, lib=lib, state_positions=state_positions)
 
 
 def decode_direct(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
                   conv_state, slot_mapping, k_cache, v_cache,
-                  state_indices=None, lib=None):
+                  state_indices=None, lib=None, state_positions=None):
     """Decode through the C entry point oracle_decode (same semantics as
     decode(); kept so both entry points are exercised)."""
     lib = lib or load()
@@ -259,8 +313,8 @@ def decode_direct(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
     k2, v2 = k.reshape(B, C), v.reshape(B, C)
     wk, wv = _u16(conv_w_k), _u16(conv_w_v)
     W = wk.shape[0]
-    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
-    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
+    gk, gv, ghs = _gammas(gamma_k, gamma_v, H)
+    pos = _positions(state_positions)
     st = _u16(conv_state).copy()
     sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
     kc, vc = _u16(k_cache).copy(), _u16(v_cache).copy()
@@ -268,10 +322,10 @@ def decode_direct(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
         state_indices, dtype=np.int32)
     zk = np.zeros((B, C), np.float64)
     zv = np.zeros((B, C), np.float64)
-    rc = lib.oracle_decode(
+    rc = lib.oracle_decode_opts(
         _p(k2, _u16p), _p(v2, _u16p), C, B, _p(wk, _u16p), _p(wv, _u16p),
-        _p(gk, _f32p), _p(gv, _f32p), float(eps), W, H, D,
-        _p(st if W > 1 else None, _u16p), _p(si, _i32p), st.shape[0],
+        _p(gk, _f32p), _p(gv, _f32p), ghs, float(eps), W, H, D,
+        _p(st if W > 1 else None, _u16p), _p(si, _i32p), _p(pos, _i64p), st.shape[0],
         _p(sm, _i64p), _p(kc, _u16p), _p(vc, _u16p), num_pages, page_size,
         page_size * C, C, D, _p(zk, _f64p), _p(zv, _f64p))
     if rc != 0:
@@ -313,7 +367,7 @@ def mx_block(values_f32, lib=None):
 
 def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                          eps, conv_state, slot_mapping, num_pages, page_size,
-                         state_indices=None, check=True, lib=None):
+                         state_indices=None, check=True, lib=None, state_positions=None):
     """The step with the MXFP8 store into dense caches: data uint8
     [num_pages, page_size, H, D], scales uint8 [num_pages, page_size, H, D/32]
     (fresh, zero-filled).  Returns dict(k_data, k_scale, v_data, v_scale,
@@ -323,10 +377,10 @@ def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
     T = k.shape[0]
     wk, wv = _u16(conv_w_k), _u16(conv_w_v)
     W, C = wk.shape
-    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
-    gv = np.ascontiguousarray(gamma_v, dtype=np.float32)
-    D = gk.shape[0]
+    D = np.asarray(gamma_k).shape[-1]
     H = C // D
+    gk, gv, ghs = _gammas(gamma_k, gamma_v, H)
+    pos = _positions(state_positions)
     k2, v2 = k.reshape(T, C), v.reshape(T, C)
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
     S = cu.shape[0] - 1
@@ -340,10 +394,10 @@ def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
     zk = np.zeros((T, C), np.float64)
     zv = np.zeros((T, C), np.float64)
     _u8p = ctypes.POINTER(ctypes.c_uint8)
-    rc = lib.oracle_prefill_varlen_mxfp8(
+    rc = lib.oracle_prefill_varlen_mxfp8_opts(
         _p(k2, _u16p), _p(v2, _u16p), C, T, _p(cu, _i32p), S, _p(wk, _u16p),
-        _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p), float(eps), W, H, D,
-        _p(st if W > 1 else None, _u16p), _p(si, _i32p), st.shape[0],
+        _p(wv, _u16p), _p(gk, _f32p), _p(gv, _f32p), ghs, float(eps), W, H, D,
+        _p(st if W > 1 else None, _u16p), _p(si, _i32p), _p(pos, _i64p), st.shape[0],
         _p(sm, _i64p), kd.ctypes.data_as(_u8p), ks.ctypes.data_as(_u8p),
         vd.ctypes.data_as(_u8p), vs.ctypes.data_as(_u8p), num_pages, page_size,
         page_size * C, C, D, _p(zk, _f64p), _p(zv, _f64p))

@@ -126,18 +126,26 @@ void oracle_conv(const uint16_t* x, int64_t row_stride, int64_t L,
  * the stated assumption).
  *   r = 1 / sqrt( (sum_d y[d]^2) / D + eps ),   z[d] = (y[d] * r) * gamma[d]
  */
-void oracle_rmsnorm(const double* y, int64_t L, int num_heads, int D,
-                    const float* gamma, double eps, double* z) {
+void oracle_rmsnorm_strided(const double* y, int64_t L, int num_heads, int D,
+                            const float* gamma, int64_t gamma_head_stride, double eps,
+                            double* z) {
   for (int64_t p = 0; p < L; ++p) {
     for (int h = 0; h < num_heads; ++h) {
       const double* yh = y + (p * num_heads + h) * (int64_t)D;
+      const float* gh = gamma + (int64_t)h * gamma_head_stride;
       double ss = 0.0;
       for (int d = 0; d < D; ++d) ss += yh[d] * yh[d];
       double r = 1.0 / sqrt(ss / (double)D + eps);
       double* zh = z + (p * num_heads + h) * (int64_t)D;
-      for (int d = 0; d < D; ++d) zh[d] = (yh[d] * r) * (double)gamma[d];
+      for (int d = 0; d < D; ++d) zh[d] = (yh[d] * r) * (double)gh[d];
     }
   }
+}
+
+/* gamma shared by all heads (gamma_head_stride 0) */
+void oracle_rmsnorm(const double* y, int64_t L, int num_heads, int D,
+                    const float* gamma, double eps, double* z) {
+  oracle_rmsnorm_strided(y, L, num_heads, D, gamma, 0, eps, z);
 }
 
 /* Address (in elements) of slot `slot`, head h, dim 0 of a paged cache. */
@@ -205,6 +213,39 @@ void oracle_state_update(const uint16_t* x, int64_t row_stride, int64_t L,
 }
 
 /*
+ * Step a5 with a ring-buffer state (a layout variant): the raw input row of
+ * position p of the sequence lives in state row p mod (W-1).  The sequence
+ * has seen pos0 tokens before this call, so its L new rows are positions
+ * pos0 .. pos0+L-1; the rows of the last min(L, W-1) of them are written,
+ * every other state row keeps its value (it still holds one of the last W-1
+ * positions).
+ */
+void oracle_state_update_ring(const uint16_t* x, int64_t row_stride, int64_t L,
+                              uint16_t* s, int64_t state_row_stride, int C, int W,
+                              int64_t pos0) {
+  const int64_t n = W - 1;
+  if (n <= 0) return;
+  const int64_t first = L > n ? L - n : 0;
+  for (int64_t q = first; q < L; ++q) {
+    const int64_t row = (pos0 + q) % n;
+    for (int c = 0; c < C; ++c) s[row * state_row_stride + c] = x[q * row_stride + c];
+  }
+}
+
+/* The W-1 rows in front of position pos0 (oldest first) from a ring state:
+ * position pos0-(W-1)+j sits in row (pos0-(W-1)+j) mod (W-1) = (pos0+j)
+ * mod (W-1); rows for positions before 0 are the zero rows a new sequence
+ * starts with. */
+static void ring_to_linear(const uint16_t* ring, int64_t state_row_stride, int W, int C2,
+                           int64_t pos0, uint16_t* lin) {
+  const int64_t n = W - 1;
+  for (int64_t j = 0; j < n; ++j) {
+    const int64_t row = (pos0 + j) % n;
+    memcpy(lin + j * C2, ring + row * state_row_stride, sizeof(uint16_t) * (size_t)C2);
+  }
+}
+
+/*
  * The whole step over a varlen batch: for each sequence i in order, for K
  * then V: conv (a1+a2) -> RMSNorm (a3) -> bf16 scatter (a4) -> state
  * update (a5).  The fused kernel reaches exactly this result; fusion only
@@ -224,18 +265,23 @@ void oracle_state_update(const uint16_t* x, int64_t row_stride, int64_t L,
  * Duplicate non-negative slots are refused (the result would depend on the
  * write order).  Returns ORACLE_OK or a negative ORACLE_ERR_*.
  */
-int oracle_prefill_varlen(
+int oracle_prefill_varlen_opts(
     const uint16_t* k, const uint16_t* v, int64_t row_stride,
     int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
     const uint16_t* conv_w_k, const uint16_t* conv_w_v, const float* gamma_k,
-    const float* gamma_v, double eps, int W, int num_heads, int D,
-    uint16_t* conv_state, const int32_t* state_indices,
-    int64_t state_pool_size, const int64_t* slot_mapping, uint16_t* k_cache,
+    const float* gamma_v, int64_t gamma_head_stride, double eps, int W,
+    int num_heads, int D, uint16_t* conv_state, const int32_t* state_indices,
+    const int64_t* state_positions, int64_t state_pool_size,
+    const int64_t* slot_mapping, uint16_t* k_cache,
     uint16_t* v_cache, int64_t num_pages, int64_t page_size,
     int64_t stride_page, int64_t stride_slot, int64_t stride_head,
     double* z_k, double* z_v) {
   if (W < 1 || num_heads < 1 || D < 1 || num_seqs < 0 || num_tokens < 0)
     return ORACLE_ERR_ARG;
+  if (gamma_head_stride != 0 && gamma_head_stride != D) return ORACLE_ERR_ARG;
+  if (state_positions)
+    for (int i = 0; i < num_seqs; ++i)
+      if (state_positions[i] < 0) return ORACLE_ERR_ARG;
   const int C = num_heads * D;
   const int64_t num_slots = num_pages * page_size;
   if (row_stride < C) return ORACLE_ERR_ARG;
@@ -290,39 +336,98 @@ int oracle_prefill_varlen(
     return ORACLE_ERR_NOMEM;
   }
 
+  /* a ring state is read through a linear copy of the rows in front of the
+     sequence (oldest first) */
+  uint16_t* lin = NULL;
+  if (state_positions && W > 1) {
+    lin = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)state_seq_stride);
+    if (!lin) {
+      free(y);
+      free(z);
+      return ORACLE_ERR_NOMEM;
+    }
+  }
+
   int status = ORACLE_OK;
   for (int i = 0; i < num_seqs; ++i) {
     const int64_t t0 = cu_seqlens[i];
     const int64_t L = cu_seqlens[i + 1] - t0;
     const int64_t si = state_indices ? state_indices[i] : i;
     uint16_t* st = conv_state ? conv_state + si * state_seq_stride : NULL;
+    const int64_t pos0 = state_positions ? state_positions[i] : 0;
+    if (lin && st) ring_to_linear(st, state_row_stride, W, 2 * C, pos0, lin);
     for (int which = 0; which < 2; ++which) { /* 0 = K, 1 = V */
       const uint16_t* x = (which == 0 ? k : v) + t0 * row_stride;
       const uint16_t* w = (which == 0 ? conv_w_k : conv_w_v);
       const float* g = (which == 0 ? gamma_k : gamma_v);
       uint16_t* cache = (which == 0 ? k_cache : v_cache);
       uint16_t* s = st ? st + (which == 0 ? 0 : C) : NULL;
+      const uint16_t* s_read = (lin && st) ? lin + (which == 0 ? 0 : C) : s;
       double* zout = (which == 0 ? z_k : z_v);
 
-      oracle_conv(x, row_stride, L, s, state_row_stride, w, W, C, y);
-      oracle_rmsnorm(y, L, num_heads, D, g, eps, z);
+      oracle_conv(x, row_stride, L, s_read, state_row_stride, w, W, C, y);
+      oracle_rmsnorm_strided(y, L, num_heads, D, g, gamma_head_stride, eps, z);
       int rc = oracle_scatter(z, L, num_heads, D, slot_mapping + t0,
                               num_slots, page_size, stride_page, stride_slot,
                               stride_head, cache);
       if (rc != ORACLE_OK) status = rc;
-      if (s) oracle_state_update(x, row_stride, L, s, state_row_stride, C, W);
+      if (s && lin) oracle_state_update_ring(x, row_stride, L, s, state_row_stride, C, W, pos0);
+      else if (s) oracle_state_update(x, row_stride, L, s, state_row_stride, C, W);
       if (zout) memcpy(zout + t0 * C, z, sizeof(double) * (size_t)(L * C));
     }
   }
+  free(lin);
   free(y);
   free(z);
   return status;
+}
+
+/* The step with gamma shared by all heads and a linear (oldest first) state. */
+int oracle_prefill_varlen(
+    const uint16_t* k, const uint16_t* v, int64_t row_stride,
+    int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
+    const uint16_t* conv_w_k, const uint16_t* conv_w_v, const float* gamma_k,
+    const float* gamma_v, double eps, int W, int num_heads, int D,
+    uint16_t* conv_state, const int32_t* state_indices,
+    int64_t state_pool_size, const int64_t* slot_mapping, uint16_t* k_cache,
+    uint16_t* v_cache, int64_t num_pages, int64_t page_size,
+    int64_t stride_page, int64_t stride_slot, int64_t stride_head,
+    double* z_k, double* z_v) {
+  return oracle_prefill_varlen_opts(k, v, row_stride, num_tokens, cu_seqlens, num_seqs,
+                                    conv_w_k, conv_w_v, gamma_k, gamma_v, 0, eps, W,
+                                    num_heads, D, conv_state, state_indices, NULL,
+                                    state_pool_size, slot_mapping, k_cache, v_cache,
+                                    num_pages, page_size, stride_page, stride_slot,
+                                    stride_head, z_k, z_v);
 }
 
 /*
  * Decode: the same step with exactly one new token per sequence
  * (cu_seqlens = 0, 1, ..., batch).
  */
+int oracle_decode_opts(const uint16_t* k, const uint16_t* v, int64_t row_stride,
+                       int batch, const uint16_t* conv_w_k,
+                       const uint16_t* conv_w_v, const float* gamma_k,
+                       const float* gamma_v, int64_t gamma_head_stride, double eps, int W,
+                       int num_heads, int D, uint16_t* conv_state,
+                       const int32_t* state_indices, const int64_t* state_positions,
+                       int64_t state_pool_size, const int64_t* slot_mapping,
+                       uint16_t* k_cache, uint16_t* v_cache, int64_t num_pages,
+                       int64_t page_size, int64_t stride_page, int64_t stride_slot,
+                       int64_t stride_head, double* z_k, double* z_v) {
+  if (batch < 0) return ORACLE_ERR_ARG;
+  int32_t* cu = (int32_t*)malloc(sizeof(int32_t) * (size_t)(batch + 1));
+  if (!cu) return ORACLE_ERR_NOMEM;
+  for (int i = 0; i <= batch; ++i) cu[i] = i;
+  int rc = oracle_prefill_varlen_opts(
+      k, v, row_stride, batch, cu, batch, conv_w_k, conv_w_v, gamma_k,
+      gamma_v, gamma_head_stride, eps, W, num_heads, D, conv_state, state_indices,
+      state_positions, state_pool_size, slot_mapping, k_cache, v_cache, num_pages,
+      page_size, stride_page, stride_slot, stride_head, z_k, z_v);
+  free(cu);
+  return rc;
+}
+
 int oracle_decode(const uint16_t* k, const uint16_t* v, int64_t row_stride,
                   int batch, const uint16_t* conv_w_k,
                   const uint16_t* conv_w_v, const float* gamma_k,
@@ -332,17 +437,10 @@ int oracle_decode(const uint16_t* k, const uint16_t* v, int64_t row_stride,
                   uint16_t* k_cache, uint16_t* v_cache, int64_t num_pages,
                   int64_t page_size, int64_t stride_page, int64_t stride_slot,
                   int64_t stride_head, double* z_k, double* z_v) {
-  if (batch < 0) return ORACLE_ERR_ARG;
-  int32_t* cu = (int32_t*)malloc(sizeof(int32_t) * (size_t)(batch + 1));
-  if (!cu) return ORACLE_ERR_NOMEM;
-  for (int i = 0; i <= batch; ++i) cu[i] = i;
-  int rc = oracle_prefill_varlen(
-      k, v, row_stride, batch, cu, batch, conv_w_k, conv_w_v, gamma_k,
-      gamma_v, eps, W, num_heads, D, conv_state, state_indices,
-      state_pool_size, slot_mapping, k_cache, v_cache, num_pages, page_size,
-      stride_page, stride_slot, stride_head, z_k, z_v);
-  free(cu);
-  return rc;
+  return oracle_decode_opts(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, 0,
+                            eps, W, num_heads, D, conv_state, state_indices, NULL,
+                            state_pool_size, slot_mapping, k_cache, v_cache, num_pages,
+                            page_size, stride_page, stride_slot, stride_head, z_k, z_v);
 }
 
 /* Vector helper for the Python side: round n doubles to bf16 bit patterns
@@ -426,13 +524,14 @@ void oracle_mx_block(const float* v, int n, uint8_t* codes, uint8_t* scale) {
  * scale caches: uint8, block (slot, h, b) at (page*stride_page +
  * off*stride_slot + h*stride_head)/32 + b (all strides multiples of 32).
  * z_k / z_v (optional) receive the unrounded double values. */
-int oracle_prefill_varlen_mxfp8(
+int oracle_prefill_varlen_mxfp8_opts(
     const uint16_t* k, const uint16_t* v, int64_t row_stride,
     int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
     const uint16_t* conv_w_k, const uint16_t* conv_w_v, const float* gamma_k,
-    const float* gamma_v, double eps, int W, int num_heads, int D,
-    uint16_t* conv_state, const int32_t* state_indices,
-    int64_t state_pool_size, const int64_t* slot_mapping, uint8_t* k_data,
+    const float* gamma_v, int64_t gamma_head_stride, double eps, int W, int num_heads,
+    int D, uint16_t* conv_state, const int32_t* state_indices,
+    const int64_t* state_positions, int64_t state_pool_size,
+    const int64_t* slot_mapping, uint8_t* k_data,
     uint8_t* k_scale, uint8_t* v_data, uint8_t* v_scale, int64_t num_pages,
     int64_t page_size, int64_t stride_page, int64_t stride_slot,
     int64_t stride_head, double* z_k, double* z_v) {
@@ -451,10 +550,10 @@ int oracle_prefill_varlen_mxfp8(
     if (!z_v) free(zv);
     return ORACLE_ERR_NOMEM;
   }
-  int rc = oracle_prefill_varlen(
+  int rc = oracle_prefill_varlen_opts(
       k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
-      gamma_k, gamma_v, eps, W, num_heads, D, conv_state, state_indices,
-      state_pool_size, slot_mapping, scratch_k, scratch_v, num_slots, 1,
+      gamma_k, gamma_v, gamma_head_stride, eps, W, num_heads, D, conv_state, state_indices,
+      state_positions, state_pool_size, slot_mapping, scratch_k, scratch_v, num_slots, 1,
       C, C, D, zk, zv);
   free(scratch_k);
   free(scratch_v);
@@ -481,6 +580,23 @@ int oracle_prefill_varlen_mxfp8(
   if (!z_k) free(zk);
   if (!z_v) free(zv);
   return rc;
+}
+
+int oracle_prefill_varlen_mxfp8(
+    const uint16_t* k, const uint16_t* v, int64_t row_stride,
+    int64_t num_tokens, const int32_t* cu_seqlens, int num_seqs,
+    const uint16_t* conv_w_k, const uint16_t* conv_w_v, const float* gamma_k,
+    const float* gamma_v, double eps, int W, int num_heads, int D,
+    uint16_t* conv_state, const int32_t* state_indices,
+    int64_t state_pool_size, const int64_t* slot_mapping, uint8_t* k_data,
+    uint8_t* k_scale, uint8_t* v_data, uint8_t* v_scale, int64_t num_pages,
+    int64_t page_size, int64_t stride_page, int64_t stride_slot,
+    int64_t stride_head, double* z_k, double* z_v) {
+  return oracle_prefill_varlen_mxfp8_opts(
+      k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v, gamma_k,
+      gamma_v, 0, eps, W, num_heads, D, conv_state, state_indices, NULL, state_pool_size,
+      slot_mapping, k_data, k_scale, v_data, v_scale, num_pages, page_size, stride_page,
+      stride_slot, stride_head, z_k, z_v);
 }
 
 /* Vector helper for the Python side: E4M3 codes of n doubles. */

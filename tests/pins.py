@@ -465,3 +465,107 @@ def pin_mxfp8_step(lib):
 
 
 ALL_PINS += [pin_e4m3_rounding, pin_mx_block, pin_mxfp8_step]
+
+
+# ------------------------------------------------------------ layout variants
+
+def pin_per_head_gamma(lib):
+    """Per-head gammas [H, D]: z equals the z of unit gammas times
+    Gamma[h, d] exactly (the oracle forms (y * r) * gamma, and y * r * 1.0
+    is y * r), for K and V separately; gammas with identical rows equal the
+    shared-gamma step bit for bit; the cache store and the state are the
+    shared-gamma ones' when the gammas agree."""
+    b = wl.make_prefill([19, 6], Hkv=3, D=64, W=4, seed=91, state="normal",
+                        page_size=8, spare_pages=1)
+    H, D = b.Hkv, b.D
+    g = torch.Generator().manual_seed(92)
+    Gk = (1 + 0.3 * torch.randn(H, D, generator=g)).numpy().astype(np.float32)
+    Gv = (1 + 0.3 * torch.randn(H, D, generator=g)).numpy().astype(np.float32)
+    ones = np.ones((H, D), np.float32)
+
+    def run(gk, gv):
+        return oracle.prefill_varlen(
+            _bits(b.k), _bits(b.v), b.cu_seqlens.numpy(), _bits(b.conv_w_k),
+            _bits(b.conv_w_v), gk, gv, b.eps, _bits(b.conv_state), b.slot_mapping.numpy(),
+            _bits(b.empty_cache()), _bits(b.empty_cache()), lib=lib)
+
+    per = run(Gk, Gv)
+    unit = run(ones, ones)
+    T = b.num_tokens
+    for z, zu, G in ((per["z_k"], unit["z_k"], Gk), (per["z_v"], unit["z_v"], Gv)):
+        want = (zu.reshape(T, H, D) * G[None].astype(np.float64)).reshape(T, H * D)
+        assert np.array_equal(z, want)
+    g0 = b.gamma_k.numpy().astype(np.float32)
+    tiled = run(np.tile(g0, (H, 1)), np.tile(b.gamma_v.numpy().astype(np.float32), (H, 1)))
+    shared = run(g0, b.gamma_v.numpy().astype(np.float32))
+    for key in ("z_k", "z_v", "k_cache", "v_cache", "conv_state"):
+        assert np.array_equal(tiled[key], shared[key]), key
+
+
+def _ring_to_linear(ring, pos):
+    """Rows of the W-1 positions in front of `pos`, oldest first, read from a
+    ring in which position p lives in row p mod (W-1) (index permutation)."""
+    n = ring.shape[0]
+    return np.stack([ring[(pos - n + j) % n] for j in range(n)]) if n else ring.copy()
+
+
+def pin_ring_state(lib):
+    """Ring-buffer state (position p in row p mod (W-1)): for random rings
+    and positions, and along chunked and decode chains, the normalised
+    values equal those of the linear state obtained by reading the ring in
+    position order, bit for bit; afterwards the ring read in the new
+    position order equals the linear step's new state; and a call rewrites
+    only the rows of its last min(L, W-1) positions."""
+    for W, lengths, seed in ((4, [1, 2, 3, 7, 0], 93), (8, [1, 5, 9, 2], 94), (2, [3, 1], 95)):
+        n = W - 1
+        b = wl.make_prefill(lengths, Hkv=2, D=64, W=W, seed=seed, state="normal",
+                            page_size=8, spare_pages=1)
+        S = b.num_seqs
+        rng = np.random.default_rng(seed)
+        pos = rng.integers(0, 50, size=S).astype(np.int64)
+        ring = _bits(b.conv_state)
+        lin = np.stack([_ring_to_linear(ring[i], pos[i]) for i in range(S)])
+        common = (_bits(b.k), _bits(b.v), b.cu_seqlens.numpy(), _bits(b.conv_w_k),
+                  _bits(b.conv_w_v), b.gamma_k.numpy(), b.gamma_v.numpy(), b.eps)
+        r_ring = oracle.prefill_varlen(*common, ring, b.slot_mapping.numpy(),
+                                       _bits(b.empty_cache()), _bits(b.empty_cache()),
+                                       state_positions=pos, lib=lib)
+        r_lin = oracle.prefill_varlen(*common, lin, b.slot_mapping.numpy(),
+                                      _bits(b.empty_cache()), _bits(b.empty_cache()), lib=lib)
+        for key in ("z_k", "z_v", "k_cache", "v_cache"):
+            assert np.array_equal(r_ring[key], r_lin[key]), (W, key)
+        cu = b.cu_seqlens.numpy()
+        for i in range(S):
+            L = int(cu[i + 1] - cu[i])
+            new = r_ring["conv_state"][i]
+            assert np.array_equal(_ring_to_linear(new, pos[i] + L), r_lin["conv_state"][i]), (W, i)
+            written = {int((pos[i] + q) % n) for q in range(max(0, L - n), L)}
+            for row in range(n):
+                if row not in written:
+                    assert np.array_equal(new[row], ring[i][row]), (W, i, row)
+    # a chain: one sequence fed in chunks and decode steps through a ring
+    # equals the one-shot linear step
+    b = wl.make_prefill([23], Hkv=2, D=64, W=4, seed=96, state="zero", page_size=8,
+                        spare_pages=1)
+    kb, vb = _bits(b.k), _bits(b.v)
+    one = oracle.prefill_varlen(kb, vb, b.cu_seqlens.numpy(), _bits(b.conv_w_k),
+                                _bits(b.conv_w_v), b.gamma_k.numpy(), b.gamma_v.numpy(), b.eps,
+                                _bits(b.conv_state), b.slot_mapping.numpy(),
+                                _bits(b.empty_cache()), _bits(b.empty_cache()), lib=lib)
+    ring = _bits(b.conv_state)
+    kc, vc = _bits(b.empty_cache()), _bits(b.empty_cache())
+    p = 0
+    for cut in (5, 1, 1, 7, 1, 8):
+        sl = slice(p, p + cut)
+        r = oracle.prefill_varlen(kb[sl], vb[sl], np.array([0, cut], np.int32),
+                                  _bits(b.conv_w_k), _bits(b.conv_w_v), b.gamma_k.numpy(),
+                                  b.gamma_v.numpy(), b.eps, ring, b.slot_mapping.numpy()[sl],
+                                  kc, vc, state_positions=np.array([p], np.int64), lib=lib)
+        assert np.array_equal(r["z_k"], one["z_k"][sl]) and np.array_equal(r["z_v"], one["z_v"][sl])
+        ring, kc, vc = r["conv_state"], r["k_cache"], r["v_cache"]
+        p += cut
+    assert np.array_equal(kc, one["k_cache"]) and np.array_equal(vc, one["v_cache"])
+    assert np.array_equal(_ring_to_linear(ring[0], p), one["conv_state"][0])
+
+
+ALL_PINS += [pin_per_head_gamma, pin_ring_state]

@@ -17,7 +17,11 @@ MUTANTS = [
     ("sign_flip", "acc += oracle_bf16_to_double", "acc -= oracle_bf16_to_double"),
     ("eps_outside_sqrt", "1.0 / sqrt(ss / (double)D + eps)", "1.0 / (sqrt(ss / (double)D) + eps)"),
     ("sum_not_mean", "1.0 / sqrt(ss / (double)D + eps)", "1.0 / sqrt(ss + eps)"),
-    ("gamma_by_head", "(double)gamma[d]", "(double)gamma[h % D]"),
+    ("gamma_by_head", "(double)gh[d]", "(double)gh[h % D]"),
+    ("gamma_head_stride_ignored", "const float* gh = gamma + (int64_t)h * gamma_head_stride;",
+     "const float* gh = gamma;"),
+    ("ring_write_row_shifted", "const int64_t row = (pos0 + q) % n;", "const int64_t row = (pos0 + q + 1) % n;"),
+    ("ring_read_ignores_position", "const int64_t row = (pos0 + j) % n;", "const int64_t row = j % n;"),
     ("state_keeps_oldest", "int64_t q = L - n + j;", "int64_t q = j;"),
     ("v_uses_k_taps", "(which == 0 ? conv_w_k : conv_w_v)", "(conv_w_k)"),
     ("v_state_in_k_half", "st + (which == 0 ? 0 : C)", "st + 0"),
