@@ -47,15 +47,18 @@ KERNEL_SOURCES = [os.path.join(ROOT, "short_conv_kv_b200", "csrc", f)
 
 # ------------------------------------------------------------------ helpers
 
-def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8, mx=False):
+def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8, mx=False, ring=False):
     """Bytes the step must move: per token K+V rows in and K+V cache rows out
     (bf16, or with the MXFP8 store one E4M3 byte per channel plus one scale
     byte per 32 channels) plus the slot; per sequence the conv_state rows in
-    and out; per launch the taps and gammas."""
+    and out (a ring-buffer state: W-1 rows in, one row out, plus the int64
+    position -- counted for one-token decode steps); per launch the taps and
+    gammas."""
     C = Hkv * D
     out = 2 * C + 2 * C // 32 if mx else 2 * C * 2
     per_token = 2 * C * 2 + out + slot_bytes
-    per_seq = 2 * (W - 1) * 2 * C * 2
+    row = 2 * C * 2
+    per_seq = (W - 1) * row + (row + 8 if ring else (W - 1) * row)
     per_launch = 2 * W * C * 2 + 2 * D * 4
     return tokens * per_token + seqs * per_seq + per_launch
 
@@ -161,6 +164,7 @@ class Workload:
     def __init__(self, name, rank):
         self.mx = name.endswith("_mx")  # MXFP8 cache store variant
         name = name[:-3] if self.mx else name
+        self.ring = name.endswith("_ring")  # ring-buffer conv_state (decode)
         self.name, self.rank = name, rank
         seed_shift = 97 * rank
         if name == "single":
@@ -180,10 +184,12 @@ class Workload:
             self.kind = "long"
             self.long = wl.long_context(seed=5000 + seed_shift)
             self.desc = "long-context chunked prefill 1,048,576 tokens in 65,536-token chunks, W=4, state carried"
-        elif name == "decode":
+        elif name in ("decode", "decode_ring"):
             self.kind = "decode"
             self.dec = wl.decode(seed=4000 + seed_shift)
             self.desc = "decode 1024 seqs x 1 token, Hkv=8, D=128, W=4, N(0,1) state, 4096-page cache"
+            if name == "decode_ring":
+                self.desc += "; ring-buffer state (one state row written per sequence)"
         else:
             raise SystemExit(f"unknown workload {name}")
 
@@ -226,7 +232,8 @@ class Workload:
             s = self.dec
             self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
             self.tokens_per_step, self.seqs_per_step = s.batch, s.batch
-            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D, mx=self.mx)
+            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D, mx=self.mx,
+                                                    ring=self.ring)
             shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
                           gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
                           k_cache=s.empty_cache().to(dev), v_cache=s.empty_cache().to(dev))
@@ -235,8 +242,12 @@ class Workload:
             states = [s.conv_state.to(dev) for _ in range(min(R, 16))]
             for r in range(R):
                 k, v, sm = s.step_inputs(r % 64)
-                self.calls_args.append(dict(k=k.to(dev), v=v.to(dev), slot_mapping=sm.to(dev),
-                                            conv_state=states[r % len(states)], **shared))
+                a = dict(k=k.to(dev), v=v.to(dev), slot_mapping=sm.to(dev),
+                         conv_state=states[r % len(states)], **shared)
+                if self.ring:
+                    pos = s.start_len.astype(np.int64) + (r % 64)
+                    a["state_positions"] = torch.from_numpy(pos).to(dev)
+                self.calls_args.append(a)
 
         if self.mx:
             # MXFP8 store: uint8 E4M3 data + E8M0 scale caches in place of
@@ -269,7 +280,7 @@ class Workload:
             return self.binding.prepare_decode(
                 a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
                 a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"], a["v_cache"],
-                stream=stream)
+                stream=stream, state_positions=a.get("state_positions"))
         return self.binding.prepare_prefill_varlen(
             a["k"], a["v"], a["cu_seqlens"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"],
             a["gamma_v"], a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"],
@@ -407,7 +418,8 @@ def time_e2e(work, steps, dev):
     step i+1's upload overlaps step i's download on the full-duplex link."""
     from short_conv_kv_b200 import binding
     a0 = work.calls_args[0]
-    in_keys = ["k", "v", "slot_mapping"] + (["cu_seqlens"] if "cu_seqlens" in a0 else [])
+    in_keys = ["k", "v", "slot_mapping"] + (["cu_seqlens"] if "cu_seqlens" in a0 else []) + \
+        (["state_positions"] if "state_positions" in a0 else [])
     NB = 2
     host_in = [{k: a0[k].cpu().pin_memory() for k in in_keys} for _ in range(NB)]
     dev_in = [{k: torch.empty_like(a0[k], device=dev) for k in in_keys} for _ in range(NB)]
@@ -450,7 +462,8 @@ def time_e2e(work, steps, dev):
             if work.kind == "decode":
                 binding.decode(di["k"], di["v"], a0["conv_w_k"], a0["conv_w_v"], a0["gamma_k"],
                                a0["gamma_v"], a0["eps"], do["conv_state"], di["slot_mapping"],
-                               do["k_cache"], do["v_cache"], stream=s_cmp)
+                               do["k_cache"], do["v_cache"], stream=s_cmp,
+                               state_positions=di.get("state_positions"))
             else:
                 binding.prefill_varlen(di["k"], di["v"], di["cu_seqlens"], a0["conv_w_k"],
                                        a0["conv_w_v"], a0["gamma_k"], a0["gamma_v"], a0["eps"],
@@ -560,7 +573,7 @@ def run_ours(args):
                          "of the written cache rows + new state, pipelined over two buffer "
                          "sets on three streams"}
     unfused = None
-    if not work.mx and not args.no_unfused:
+    if not work.mx and not work.ring and not args.no_unfused:
         Ku = min(K, 50)
         un_ms = max_over_ranks(time_unfused(work, Ku, Wu, dev), world)
         T, C = work.tokens_per_step, work.Hkv * work.D
@@ -689,7 +702,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="single",
-                    choices=["single", "varlen", "decode", "long", "wsweep2", "wsweep4", "wsweep8",
+                    choices=["single", "varlen", "decode", "decode_ring", "long", "wsweep2",
+                             "wsweep4", "wsweep8",
                              "single_mx", "varlen_mx", "decode_mx", "long_mx", "wsweep2_mx",
                              "wsweep4_mx", "wsweep8_mx"])
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -227,6 +227,73 @@ SCONV_KV_API int sconv_kv_decode_mxfp8(
     void* stream);
 
 /*
+ * Layout variants (the _ex entry points; NULL options = the defaults of the
+ * entry points above).
+ *
+ *  gamma_head_stride  elements between consecutive heads' gammas: 0 (the
+ *                     default) = gamma_k/v are [head_dim], shared by every
+ *                     head; head_dim = per-head gammas [num_kv_heads,
+ *                     head_dim].  Other values: SCONV_KV_ERR_SHAPE.
+ *  state_positions    NULL (default): conv_state holds each sequence's last
+ *                     W-1 raw rows oldest first, all rewritten by every
+ *                     call.  Otherwise device int64 [num_seqs] (decode:
+ *                     [batch]), the number of tokens sequence i has seen
+ *                     before this call, and conv_state is a ring: the raw
+ *                     row of position p lives in row p mod (W-1).  A call
+ *                     then writes only the rows of its sequence's last
+ *                     min(L, W-1) positions (one row per decode step instead
+ *                     of W-1); a new sequence starts at position 0 with
+ *                     zeroed rows, as in the linear layout.  A negative
+ *                     position skips the sequence and sets
+ *                     SCONV_KV_FLAG_STATE_INDEX.
+ *
+ * The pages fix neither (their norm is only "normalization" and the state
+ * pool's layout is not given); both are layouts a serving runtime may use.
+ */
+typedef struct sconv_kv_options_t {
+  int64_t gamma_head_stride;
+  const int64_t* state_positions;
+} sconv_kv_options_t;
+
+SCONV_KV_API int sconv_kv_prefill_varlen_ex(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, const sconv_kv_options_t* options,
+    int* err_flag, void* stream);
+
+SCONV_KV_API int sconv_kv_decode_ex(
+    const void* k, const void* v, int64_t row_stride, int batch,
+    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+    void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, const sconv_kv_options_t* options,
+    int* err_flag, void* stream);
+
+SCONV_KV_API int sconv_kv_prefill_varlen_mxfp8_ex(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout,
+    const sconv_kv_options_t* options, int* err_flag, void* stream);
+
+SCONV_KV_API int sconv_kv_decode_mxfp8_ex(
+    const void* k, const void* v, int64_t row_stride, int batch,
+    const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+    const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+    void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout,
+    const sconv_kv_options_t* options, int* err_flag, void* stream);
+
+/*
  * Unfused stages.  The same step as four separate passes over HBM, each
  * with its intermediate in bf16: the chain that the fused entry points
  * replace ("SGLang and Miles announce day-0 Inkling support", aib.vote

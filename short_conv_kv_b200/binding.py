@@ -30,6 +30,11 @@ class CacheLayout(ctypes.Structure):
         "stride_slot", "stride_head", "bytes_per_cache")]
 
 
+class Options(ctypes.Structure):
+    """sconv_kv_options_t: per-head gamma stride and ring-state positions."""
+    _fields_ = [("gamma_head_stride", ctypes.c_int64), ("state_positions", ctypes.c_void_p)]
+
+
 class SconvKVError(RuntimeError):
     def __init__(self, code, where):
         msg = _lib.sconv_kv_strerror(code).decode()
@@ -66,6 +71,23 @@ def _load(path):
         vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
         vp, vp, vp, vp, lp, ip, vp]
     lib.sconv_kv_decode_mxfp8.restype = i32
+    op = ctypes.POINTER(Options)
+    lib.sconv_kv_prefill_varlen_ex.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp,
+        i64, vp, vp, vp, lp, op, ip, vp]
+    lib.sconv_kv_prefill_varlen_ex.restype = i32
+    lib.sconv_kv_decode_ex.argtypes = [
+        vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
+        vp, vp, lp, op, ip, vp]
+    lib.sconv_kv_decode_ex.restype = i32
+    lib.sconv_kv_prefill_varlen_mxfp8_ex.argtypes = [
+        vp, vp, i64, i64, vp, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp,
+        i64, vp, vp, vp, vp, vp, lp, op, ip, vp]
+    lib.sconv_kv_prefill_varlen_mxfp8_ex.restype = i32
+    lib.sconv_kv_decode_mxfp8_ex.argtypes = [
+        vp, vp, i64, i32, vp, vp, vp, vp, f32, i32, i32, i32, vp, vp, i64, vp,
+        vp, vp, vp, vp, lp, op, ip, vp]
+    lib.sconv_kv_decode_mxfp8_ex.restype = i32
     lib.sconv_kv_stage_conv.argtypes = [
         vp, vp, i64, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp, i64, vp, ip, vp]
     lib.sconv_kv_stage_conv.restype = i32
@@ -137,6 +159,21 @@ def _stream(stream):
     return int(stream)
 
 
+def _options(gamma_k, state_positions):
+    """Options struct for the _ex entry points, or None for the defaults
+    (gamma [D] shared by every head, linear state).  gamma [Hkv, D] selects
+    per-head gammas; state_positions (int64 [S] on the device) a ring state."""
+    per_head = gamma_k is not None and gamma_k.dim() == 2
+    if not per_head and state_positions is None:
+        return None
+    if state_positions is not None and state_positions.dtype != torch.int64:
+        raise TypeError("state_positions must be int64")
+    o = Options()
+    o.gamma_head_stride = gamma_k.shape[-1] if per_head else 0
+    o.state_positions = _ptr(state_positions)
+    return o
+
+
 def _rows(x, name):
     """(pointer, row_stride) of a [T, Hkv, D] or [T, Hkv*D] bf16 view whose
     channels are contiguous."""
@@ -154,7 +191,7 @@ def _rows(x, name):
 def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                    eps, conv_state, slot_mapping, k_cache, v_cache,
                    state_indices=None, err_flag=None, stream=None,
-                   layout=None):
+                   layout=None, state_positions=None):
     """Fused ShortConv K/V step over a packed varlen batch, on the GPU.
 
     k, v: bf16 [T, Hkv, D] (rows may be strided slices); cu_seqlens int32
@@ -174,19 +211,24 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
     if v_cache.stride() != k_cache.stride() or v_cache.shape != k_cache.shape:
         raise ValueError("k_cache and v_cache must have the same shape and strides")
     pool = conv_state.shape[0] if conv_state is not None else 0
-    rc = _lib.sconv_kv_prefill_varlen(
-        kp, vp, rs, T, _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
-        _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
-        float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
-        _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_cache),
-        _ptr(v_cache), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    args = (kp, vp, rs, T, _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+            _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
+            float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
+            _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_cache),
+            _ptr(v_cache), ctypes.byref(lay))
+    opts = _options(gamma_k, state_positions)
+    if opts is None:
+        rc = _lib.sconv_kv_prefill_varlen(*args, _ptr(err_flag), _stream(stream))
+    else:
+        rc = _lib.sconv_kv_prefill_varlen_ex(*args, ctypes.byref(opts), _ptr(err_flag),
+                                             _stream(stream))
     if rc != OK:
         raise SconvKVError(rc, "sconv_kv_prefill_varlen")
 
 
 def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
            slot_mapping, k_cache, v_cache, state_indices=None, err_flag=None,
-           stream=None, layout=None):
+           stream=None, layout=None, state_positions=None):
     """Fused ShortConv K/V decode step: one new token per sequence
     (k, v: bf16 [B, Hkv, D]); same other arguments as prefill_varlen."""
     kp, rs = _rows(k, "k")
@@ -198,12 +240,15 @@ def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
     H, D = k_cache.shape[2], k_cache.shape[3]
     lay = layout if layout is not None else layout_of(k_cache)
     pool = conv_state.shape[0] if conv_state is not None else 0
-    rc = _lib.sconv_kv_decode(
-        kp, vp, rs, B, _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
-        _ptr(gamma_v), float(eps), W, H, D,
-        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
-        _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
-        _ptr(err_flag), _stream(stream))
+    args = (kp, vp, rs, B, _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+            _ptr(gamma_v), float(eps), W, H, D,
+            _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay))
+    opts = _options(gamma_k, state_positions)
+    if opts is None:
+        rc = _lib.sconv_kv_decode(*args, _ptr(err_flag), _stream(stream))
+    else:
+        rc = _lib.sconv_kv_decode_ex(*args, ctypes.byref(opts), _ptr(err_flag), _stream(stream))
     if rc != OK:
         raise SconvKVError(rc, "sconv_kv_decode")
 
@@ -230,7 +275,7 @@ def _mx_layout(k_data, k_scale, v_data, v_scale):
 
 def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                          eps, conv_state, slot_mapping, k_data, k_scale, v_data, v_scale,
-                         state_indices=None, err_flag=None, stream=None):
+                         state_indices=None, err_flag=None, stream=None, state_positions=None):
     """The fused step with the block-scaled MXFP8 cache store (E4M3 codes in
     k_data/v_data, one E8M0 scale byte per 32 channels in k_scale/v_scale)."""
     kp, rs = _rows(k, "k")
@@ -241,19 +286,23 @@ def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
     W = conv_w_k.shape[0]
     H, D = k_data.shape[2], k_data.shape[3]
     pool = conv_state.shape[0] if conv_state is not None else 0
-    rc = _lib.sconv_kv_prefill_varlen_mxfp8(
-        kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
-        _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v), float(eps), W, H, D,
-        _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(slot_mapping),
-        _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale), ctypes.byref(lay),
-        _ptr(err_flag), _stream(stream))
+    args = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+            _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v), float(eps), W, H, D,
+            _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(slot_mapping),
+            _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale), ctypes.byref(lay))
+    opts = _options(gamma_k, state_positions)
+    if opts is None:
+        rc = _lib.sconv_kv_prefill_varlen_mxfp8(*args, _ptr(err_flag), _stream(stream))
+    else:
+        rc = _lib.sconv_kv_prefill_varlen_mxfp8_ex(*args, ctypes.byref(opts), _ptr(err_flag),
+                                                   _stream(stream))
     if rc != OK:
         raise SconvKVError(rc, "sconv_kv_prefill_varlen_mxfp8")
 
 
 def decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
                  slot_mapping, k_data, k_scale, v_data, v_scale, state_indices=None,
-                 err_flag=None, stream=None):
+                 err_flag=None, stream=None, state_positions=None):
     """Decode step with the MXFP8 cache store (one new token per sequence)."""
     kp, rs = _rows(k, "k")
     vp, rs_v = _rows(v, "v")
@@ -263,11 +312,16 @@ def decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
     W = conv_w_k.shape[0]
     H, D = k_data.shape[2], k_data.shape[3]
     pool = conv_state.shape[0] if conv_state is not None else 0
-    rc = _lib.sconv_kv_decode_mxfp8(
-        kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
-        _ptr(gamma_v), float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
-        _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
-        _ptr(v_data), _ptr(v_scale), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
+    args = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+            _ptr(gamma_v), float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
+            _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
+            _ptr(v_data), _ptr(v_scale), ctypes.byref(lay))
+    opts = _options(gamma_k, state_positions)
+    if opts is None:
+        rc = _lib.sconv_kv_decode_mxfp8(*args, _ptr(err_flag), _stream(stream))
+    else:
+        rc = _lib.sconv_kv_decode_mxfp8_ex(*args, ctypes.byref(opts), _ptr(err_flag),
+                                           _stream(stream))
     if rc != OK:
         raise SconvKVError(rc, "sconv_kv_decode_mxfp8")
 
@@ -310,19 +364,24 @@ def prepare_prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k,
 
 def prepare_decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
                    conv_state, slot_mapping, k_cache, v_cache,
-                   state_indices=None, err_flag=None, stream=None):
+                   state_indices=None, err_flag=None, stream=None, state_positions=None):
     kp, rs = _rows(k, "k")
     vp, _ = _rows(v, "v")
     W = conv_w_k.shape[0]
     H, D = k_cache.shape[2], k_cache.shape[3]
     lay = layout_of(k_cache)
     pool = conv_state.shape[0] if conv_state is not None else 0
-    args = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v),
+    opts = _options(gamma_k, state_positions)
+    head = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v),
             _ptr(gamma_k), _ptr(gamma_v), ctypes.c_float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
-            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
-            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
-    return PreparedCall("sconv_kv_decode", args, keep_alive=(lay,))
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay))
+    if opts is None:
+        return PreparedCall("sconv_kv_decode", head + (_ptr(err_flag), _stream(stream)),
+                            keep_alive=(lay,))
+    return PreparedCall("sconv_kv_decode_ex",
+                        head + (ctypes.byref(opts), _ptr(err_flag), _stream(stream)),
+                        keep_alive=(lay, opts))
 
 
 def prepare_prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,

@@ -45,6 +45,13 @@ struct StepParams {
   uint8_t* v_data;
   uint8_t* k_scale;
   uint8_t* v_scale;
+  // layout variants: elements between heads' gammas (0 = one gamma [D]
+  // shared by all heads), and the ring-buffer state's positions (nullptr =
+  // linear state, oldest row first; else the raw row of position p of
+  // sequence i lives in state row p mod (W-1), and state_pos[i] is the
+  // number of tokens the sequence has seen before this call)
+  int64_t gamma_hs;
+  const int64_t* state_pos;
 };
 
 // Flag bits (same values as the public SCONV_KV_FLAG_*).

@@ -14,7 +14,8 @@
 //   - the new state is exactly stage rows 1..W-1 (old rows 1..W-2, then the
 //     new row), so thread 0 writes it back with bulk shared->global copies
 //     over the rows just read -- the state update never passes through
-//     registers;
+//     registers (with a ring-buffer state only the new row is written, into
+//     the row of the oldest position);
 //   - every thread convolves its 8 channels over the W rows, reduces the
 //     head's sum of squares by xor shuffles, and stores its 16 bytes of the
 //     normalised bf16 row into the cache slot.
@@ -58,10 +59,13 @@ __device__ __forceinline__ void bulk_wait_all() {
 template <int W>
 constexpr int decode_ctas_per_sm() { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
 
-template <int W, int D, bool MX>
+template <int W, int D, bool MX, bool LV>
 __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     decode_tma_kernel(const StepParams P, const DecGeom Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // layout variants only in the LV instances (compile-time defaults elsewhere)
+  const int64_t gamma_hs = LV ? P.gamma_hs : 0;
+  const int64_t* const state_pos = LV ? P.state_pos : nullptr;
   constexpr int G = D / 8;
   const int B = P.num_seqs;
   const int NS = Gm.stages;
@@ -83,7 +87,9 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
   uint64_t* empty = full + NS;
   long long* s_off = reinterpret_cast<long long*>(empty + NS);  // cache row offset or -1
   long long* s_si = s_off + kDecMaxSeqs;                        // state row, -1 = skip
-  volatile int* abort = reinterpret_cast<volatile int*>(s_si + kDecMaxSeqs);
+  // ring-buffer state: row of the window's oldest position (-1 = linear)
+  int* s_rot = reinterpret_cast<int*>(s_si + kDecMaxSeqs);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_rot + kDecMaxSeqs);
 
   const int lane = threadIdx.x & 31;
   const int b0 = blockIdx.x;
@@ -102,14 +108,18 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
   for (int q = threadIdx.x; q < nq; q += blockDim.x) {
     const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
     int64_t si = b;
+    int rot = -1;
     if (W > 1) {
       si = P.state_indices ? static_cast<int64_t>(P.state_indices[b]) : b;
-      if (si < 0 || si >= P.pool) {
+      const int64_t pos = state_pos ? state_pos[b] : 0;
+      if (si < 0 || si >= P.pool || pos < 0) {
         if (report) raise_flag(P.err, kFlagStateIndex);
         si = -1;
       }
+      if (state_pos) rot = static_cast<int>(pos % (W - 1));
     }
     s_si[q] = si;
+    s_rot[q] = rot;
     s_off[q] = slot_row_offset(P, P.slots[b], report);
   }
   if (nq == 0) return;
@@ -141,15 +151,20 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     if (kn) bulk_g2s(xd, P.k + b * P.row_stride + g0 * 8, kn * 16, &full[st]);
     if (vn) bulk_g2s(xd + kn * 16, P.v + b * P.row_stride + (vg0 - half) * 8, vn * 16, &full[st]);
   };
-  // new state rows 0..W-2 <- stage rows 1..W-1
+  // linear state: new rows 0..W-2 <- stage rows 1..W-1; ring state: the
+  // new row (stage row W-1) <- into row rot, the slot of its position (the
+  // window's oldest position, no longer needed), and nothing else moves
   auto write_state = [&](int q) {
     const long long si = s_si[q];
-    const unsigned char* src = ring + static_cast<size_t>(q % NS) * stage_bytes + row_bytes;
-    uint16_t* sp = P.state + si * (W - 1) * srow;
+    const int rot = LV ? s_rot[q] : -1;
+    const unsigned char* src = ring + static_cast<size_t>(q % NS) * stage_bytes +
+                               (rot < 0 ? row_bytes : (W - 1) * row_bytes);
+    uint16_t* sp = P.state + si * (W - 1) * srow + (rot < 0 ? 0 : rot * srow);
+    const int nrow = rot < 0 ? W - 1 : 1;
     if (full_slice) {
-      bulk_s2g(sp, src, (W - 1) * row_bytes);
+      bulk_s2g(sp, src, nrow * row_bytes);
     } else {
-      for (int r = 0; r < W - 1; ++r) {
+      for (int r = 0; r < nrow; ++r) {
         if (kn) bulk_s2g(sp + r * srow + g0 * 8, src + r * row_bytes, kn * 16);
         if (vn)
           bulk_s2g(sp + r * srow + P.C + (vg0 - half) * 8, src + r * row_bytes + kn * 16,
@@ -198,7 +213,7 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
   uint4 twp[W];
 #pragma unroll
   for (int j = 0; j < W; ++j) twp[j] = ld_ro(w + static_cast<int64_t>(j) * P.C);
-  const float* gam = (isv ? P.gamma_v : P.gamma_k) + d0;  // read per sequence (L1)
+  const float* gam = (isv ? P.gamma_v : P.gamma_k) + (c0 / D) * gamma_hs + d0;  // per sequence
 
   for (int q = 0; q < nq; ++q) {
     const int st = q % NS;
@@ -216,10 +231,13 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
       const unsigned char* stage =
           ring + static_cast<size_t>(st) * stage_bytes + (active ? lg : 0) * 16;
       float2 acc[4];
+      // ring state: tap j reads row (rot + j) mod (W-1)
+      const int rot = (LV && W > 1) ? max(s_rot[q], 0) : 0;
 #pragma unroll
       for (int j = 0; j < W; ++j) {
         float2 rf[4], tw[4];
-        unpack8(*reinterpret_cast<const uint4*>(stage + j * row_bytes), rf);
+        const int row = j == W - 1 ? j : (rot + j < W - 1 ? rot + j : rot + j - (W - 1));
+        unpack8(*reinterpret_cast<const uint4*>(stage + row * row_bytes), rf);
         unpack8(twp[j], tw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] = j == 0 ? fmul2(tw[e], rf[e]) : ffma2(tw[e], rf[e], acc[e]);

@@ -173,11 +173,16 @@ __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 
   }
 }
 
-template <int W, int D, int MINB, bool MX>
+template <int W, int D, int MINB, bool MX, bool LV>
 __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int R = kTmaRows;
+  // layout variants (per-head gamma stride, ring-buffer state) only in the
+  // LV instances: elsewhere these fold to the defaults at compile time, so
+  // the default path carries no extra live values
+  const int64_t gamma_hs = LV ? P.gamma_hs : 0;
+  const int64_t* const state_pos = LV ? P.state_pos : nullptr;
   const int S = P.num_seqs;
   const int T = static_cast<int>(P.num_tokens);
   const int NS = Gm.stages;
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
                                              kTmaGammaBytes) + threadIdx.x * 8;
   float2 gm[4];
   {
-    const float* gam = (isv ? P.gamma_v : P.gamma_k) + d0;
+    const float* gam = (isv ? P.gamma_v : P.gamma_k) + (c0 / D) * gamma_hs + d0;
     const float4 a = __ldg(reinterpret_cast<const float4*>(gam));
     const float4 b = __ldg(reinterpret_cast<const float4*>(gam) + 1);
     if constexpr (gamma_in_smem<W>()) {
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     si = i;
     if constexpr (W > 1) {
       si = P.state_indices ? static_cast<int64_t>(P.state_indices[i]) : i;
-      if (si < 0 || si >= P.pool) {
+      if (si < 0 || si >= P.pool || (state_pos && state_pos[i] < 0)) {
         if (report) raise_flag(P.err, kFlagStateIndex);
         return false;
       }
@@ -438,26 +443,42 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     if constexpr (W > 1) {
       const int a = cu(i), e = cu(i + 1);
       uint16_t* st = P.state + si * (W - 1) * srow + st_chan;
+      // ring state: position p in row p mod (W-1); the window's oldest row
+      // (position pos0-(W-1)) sits in row pos0 mod (W-1)
+      const int rot = state_pos ? static_cast<int>(state_pos[i] % (W - 1)) : 0;
       uint4 hb[W - 1];
 #pragma unroll
-      for (int j = 0; j < W - 1; ++j)
-        hb[j] = active ? *reinterpret_cast<const uint4*>(st + j * srow) : make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < W - 1; ++j) {
+        const int row = rot + j < W - 1 ? rot + j : rot + j - (W - 1);
+        hb[j] = active ? *reinterpret_cast<const uint4*>(st + row * srow) : make_uint4(0, 0, 0, 0);
+      }
       if (active) {
         const int L = e - a;
         const uint16_t* xs = xbase + static_cast<int64_t>(a) * P.row_stride;
+        if (state_pos) {
+          // ring: only the rows of the last min(L, W-1) positions change
 #pragma unroll
-        for (int j = 0; j < W - 1; ++j) {
-          const int q = L - (W - 1) + j;  // row of (old state ++ sequence)
-          uint4 r;
-          if (q >= 0) {
-            r = ld_ro(xs + static_cast<int64_t>(q) * P.row_stride);
-          } else {
-            r = hb[0];
-#pragma unroll
-            for (int m = 1; m < W - 1; ++m)
-              if (m == W - 1 + q) r = hb[m];
+          for (int j = 0; j < W - 1; ++j) {
+            const int q = L - (W - 1) + j;
+            if (q >= 0)
+              *reinterpret_cast<uint4*>(st + ((rot + q) % (W - 1)) * srow) =
+                  ld_ro(xs + static_cast<int64_t>(q) * P.row_stride);
           }
-          *reinterpret_cast<uint4*>(st + j * srow) = r;
+        } else {
+#pragma unroll
+          for (int j = 0; j < W - 1; ++j) {
+            const int q = L - (W - 1) + j;  // row of (old state ++ sequence)
+            uint4 r;
+            if (q >= 0) {
+              r = ld_ro(xs + static_cast<int64_t>(q) * P.row_stride);
+            } else {
+              r = hb[0];
+#pragma unroll
+              for (int m = 1; m < W - 1; ++m)
+                if (m == W - 1 + q) r = hb[m];
+            }
+            *reinterpret_cast<uint4*>(st + j * srow) = r;
+          }
         }
       }
 #pragma unroll

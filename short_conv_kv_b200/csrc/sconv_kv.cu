@@ -55,23 +55,39 @@ struct Pick {
     }
   }
 };
-// bf16 store / MXFP8 store instances of each kernel
-template <int W, int D>
-struct DecodeK {
-  static DecFn get() { return sconv::decode_tma_kernel<W, D, false>; }
+// Kernel instances: bf16 or MXFP8 store (MX), without or with the layout
+// variants (LV: per-head gamma stride, ring-buffer state).
+template <bool MX, bool LV>
+struct DecodeKs {
+  template <int W, int D>
+  struct K {
+    static DecFn get() { return sconv::decode_tma_kernel<W, D, MX, LV>; }
+  };
 };
-template <int W, int D>
-struct DecodeKMx {
-  static DecFn get() { return sconv::decode_tma_kernel<W, D, true>; }
+template <bool MX, bool LV>
+struct PrefillKs {
+  template <int W, int D>
+  struct K {
+    static TmaFn get() {
+      return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), MX, LV>;
+    }
+  };
 };
-template <int W, int D>
-struct PrefillK {
-  static TmaFn get() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), false>; }
-};
-template <int W, int D>
-struct PrefillKMx {
-  static TmaFn get() { return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), true>; }
-};
+bool uses_layout_variants(const sconv_kv_options_t* opts) {
+  return opts && (opts->gamma_head_stride != 0 || opts->state_positions != nullptr);
+}
+TmaFn pick_prefill(int W, int D, bool mx, bool lv) {
+  if (mx) return lv ? Pick<TmaFn, PrefillKs<true, true>::K>::get(W, D)
+                    : Pick<TmaFn, PrefillKs<true, false>::K>::get(W, D);
+  return lv ? Pick<TmaFn, PrefillKs<false, true>::K>::get(W, D)
+            : Pick<TmaFn, PrefillKs<false, false>::K>::get(W, D);
+}
+DecFn pick_decode(int W, int D, bool mx, bool lv) {
+  if (mx) return lv ? Pick<DecFn, DecodeKs<true, true>::K>::get(W, D)
+                    : Pick<DecFn, DecodeKs<true, false>::K>::get(W, D);
+  return lv ? Pick<DecFn, DecodeKs<false, true>::K>::get(W, D)
+            : Pick<DecFn, DecodeKs<false, false>::K>::get(W, D);
+}
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
@@ -181,6 +197,18 @@ int validate_common(const void* k, const void* v, int64_t row_stride,
   return SCONV_KV_OK;
 }
 
+// Layout variants (per-head gamma stride, ring-buffer state positions).
+int apply_options(const sconv_kv_options_t* opts, int head_dim, StepParams* P) {
+  P->gamma_hs = 0;
+  P->state_pos = nullptr;
+  if (!opts) return SCONV_KV_OK;
+  if (opts->gamma_head_stride != 0 && opts->gamma_head_stride != head_dim)
+    return SCONV_KV_ERR_SHAPE;
+  P->gamma_hs = opts->gamma_head_stride;
+  P->state_pos = opts->state_positions;
+  return SCONV_KV_OK;
+}
+
 // Launch with programmatic stream serialisation: the kernel may start
 // while the previous kernel in the stream drains; it waits for that kernel
 // (griddepcontrol.wait) before touching global memory.
@@ -215,7 +243,7 @@ int prefill_impl(
     const int32_t* state_indices, int64_t state_pool_size,
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
     const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream, bool mx,
-    uint8_t* k_scale, uint8_t* v_scale) {
+    uint8_t* k_scale, uint8_t* v_scale, const sconv_kv_options_t* opts) {
   // an empty call enqueues nothing; its pointers are not examined (empty
   // tensors may have NULL data pointers)
   if (num_seqs < 0 || num_tokens < 0 || num_tokens > INT32_MAX) return SCONV_KV_ERR_SHAPE;
@@ -225,8 +253,10 @@ int prefill_impl(
                            num_kv_heads, head_dim, conv_state, state_pool_size,
                            slot_mapping, k_cache, v_cache, layout, &P, k_scale, v_scale, mx);
   if (rc != SCONV_KV_OK) return rc;
+  rc = apply_options(opts, head_dim, &P);
+  if (rc != SCONV_KV_OK) return rc;
   if (!cu_seqlens) return SCONV_KV_ERR_NULL;
-  TmaFn fn = mx ? Pick<TmaFn, PrefillKMx>::get(W, head_dim) : Pick<TmaFn, PrefillK>::get(W, head_dim);
+  TmaFn fn = pick_prefill(W, head_dim, mx, uses_layout_variants(opts));
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
 
   P.num_tokens = num_tokens;
@@ -278,7 +308,7 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
                 void* conv_state, const int32_t* state_indices, int64_t state_pool_size,
                 const int64_t* slot_mapping, void* k_cache, void* v_cache,
                 const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream, bool mx,
-                uint8_t* k_scale, uint8_t* v_scale) {
+                uint8_t* k_scale, uint8_t* v_scale, const sconv_kv_options_t* opts) {
   if (batch < 0) return SCONV_KV_ERR_SHAPE;
   if (batch == 0) return SCONV_KV_OK;  // nothing enqueued, pointers not examined
   StepParams P;
@@ -286,7 +316,9 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
                            num_kv_heads, head_dim, conv_state, state_pool_size,
                            slot_mapping, k_cache, v_cache, layout, &P, k_scale, v_scale, mx);
   if (rc != SCONV_KV_OK) return rc;
-  DecFn fn = mx ? Pick<DecFn, DecodeKMx>::get(W, head_dim) : Pick<DecFn, DecodeK>::get(W, head_dim);
+  rc = apply_options(opts, head_dim, &P);
+  if (rc != SCONV_KV_OK) return rc;
+  DecFn fn = pick_decode(W, head_dim, mx, uses_layout_variants(opts));
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
   P.num_tokens = batch;
   P.num_seqs = batch;
@@ -315,7 +347,8 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
   G.ctas = static_cast<int>(ctas);
   if (ctas_y > 65535) return SCONV_KV_ERR_SHAPE;
   const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages +
-                      2 * sconv::kDecMaxSeqs * sizeof(long long) + 16;
+                      2 * sconv::kDecMaxSeqs * sizeof(long long) +
+                      sconv::kDecMaxSeqs * sizeof(int) + 16;
   if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
     snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
     return SCONV_KV_ERR_CUDA;
@@ -462,7 +495,7 @@ int sconv_kv_prefill_varlen(
   return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
                       gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
                       state_indices, state_pool_size, slot_mapping, k_cache, v_cache, layout,
-                      err_flag, stream, false, nullptr, nullptr);
+                      err_flag, stream, false, nullptr, nullptr, nullptr);
 }
 
 int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
@@ -475,7 +508,7 @@ int sconv_kv_decode(const void* k, const void* v, int64_t row_stride, int batch,
   return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
                      num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
                      slot_mapping, k_cache, v_cache, layout, err_flag, stream, false, nullptr,
-                     nullptr);
+                     nullptr, nullptr);
 }
 
 int sconv_kv_prefill_varlen_mxfp8(
@@ -489,7 +522,7 @@ int sconv_kv_prefill_varlen_mxfp8(
   return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
                       gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
                       state_indices, state_pool_size, slot_mapping, k_data, v_data, layout,
-                      err_flag, stream, true, k_scale, v_scale);
+                      err_flag, stream, true, k_scale, v_scale, nullptr);
 }
 
 int sconv_kv_decode_mxfp8(const void* k, const void* v, int64_t row_stride, int batch,
@@ -502,7 +535,65 @@ int sconv_kv_decode_mxfp8(const void* k, const void* v, int64_t row_stride, int 
   return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
                      num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
                      slot_mapping, k_data, v_data, layout, err_flag, stream, true, k_scale,
-                     v_scale);
+                     v_scale, nullptr);
+}
+
+int sconv_kv_prefill_varlen_ex(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_cache, void* v_cache,
+    const sconv_kv_cache_layout_t* layout, const sconv_kv_options_t* options,
+    int* err_flag, void* stream) {
+  return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                      gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
+                      state_indices, state_pool_size, slot_mapping, k_cache, v_cache, layout,
+                      err_flag, stream, false, nullptr, nullptr, options);
+}
+
+int sconv_kv_decode_ex(const void* k, const void* v, int64_t row_stride, int batch,
+                       const void* conv_w_k, const void* conv_w_v, const float* gamma_k,
+                       const float* gamma_v, float eps, int W, int num_kv_heads, int head_dim,
+                       void* conv_state, const int32_t* state_indices,
+                       int64_t state_pool_size, const int64_t* slot_mapping, void* k_cache,
+                       void* v_cache, const sconv_kv_cache_layout_t* layout,
+                       const sconv_kv_options_t* options, int* err_flag, void* stream) {
+  return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
+                     num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
+                     slot_mapping, k_cache, v_cache, layout, err_flag, stream, false, nullptr,
+                     nullptr, options);
+}
+
+int sconv_kv_prefill_varlen_mxfp8_ex(
+    const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+    const void* conv_w_v, const float* gamma_k, const float* gamma_v,
+    float eps, int W, int num_kv_heads, int head_dim, void* conv_state,
+    const int32_t* state_indices, int64_t state_pool_size,
+    const int64_t* slot_mapping, void* k_data, uint8_t* k_scale, void* v_data,
+    uint8_t* v_scale, const sconv_kv_cache_layout_t* layout,
+    const sconv_kv_options_t* options, int* err_flag, void* stream) {
+  return prefill_impl(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                      gamma_k, gamma_v, eps, W, num_kv_heads, head_dim, conv_state,
+                      state_indices, state_pool_size, slot_mapping, k_data, v_data, layout,
+                      err_flag, stream, true, k_scale, v_scale, options);
+}
+
+int sconv_kv_decode_mxfp8_ex(const void* k, const void* v, int64_t row_stride, int batch,
+                             const void* conv_w_k, const void* conv_w_v,
+                             const float* gamma_k, const float* gamma_v, float eps, int W,
+                             int num_kv_heads, int head_dim, void* conv_state,
+                             const int32_t* state_indices, int64_t state_pool_size,
+                             const int64_t* slot_mapping, void* k_data, uint8_t* k_scale,
+                             void* v_data, uint8_t* v_scale,
+                             const sconv_kv_cache_layout_t* layout,
+                             const sconv_kv_options_t* options, int* err_flag, void* stream) {
+  return decode_impl(k, v, row_stride, batch, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, W,
+                     num_kv_heads, head_dim, conv_state, state_indices, state_pool_size,
+                     slot_mapping, k_data, v_data, layout, err_flag, stream, true, k_scale,
+                     v_scale, options);
 }
 
 int sconv_kv_unfused_step_noalloc(
