@@ -247,12 +247,26 @@ SCONV_KV_API int sconv_kv_decode_mxfp8(
  *                     position skips the sequence and sets
  *                     SCONV_KV_FLAG_STATE_INDEX.
  *
+ *  wait_timeout_ns    longest time a pipeline wait inside the kernels may
+ *                     take before the kernel gives up, lets the copies it
+ *                     has issued land, sets SCONV_KV_FLAG_TIMEOUT and
+ *                     returns with its output incomplete (<= 0: 1 s).  A
+ *                     short limit exercises that path without any fault.
+ *  withhold_first_copy  testing only (0 in normal use): nonzero makes every
+ *                     CTA skip the copy of its first chunk (decode: of its
+ *                     first sequence), so the waits on it run out after
+ *                     wait_timeout_ns and the timeout path above runs: a
+ *                     wait on something that nothing completes, with no
+ *                     fault.  The output of such a call is incomplete.
+ *
  * The pages fix neither (their norm is only "normalization" and the state
  * pool's layout is not given); both are layouts a serving runtime may use.
  */
 typedef struct sconv_kv_options_t {
   int64_t gamma_head_stride;
   const int64_t* state_positions;
+  int64_t wait_timeout_ns;
+  int64_t withhold_first_copy;
 } sconv_kv_options_t;
 
 SCONV_KV_API int sconv_kv_prefill_varlen_ex(

@@ -32,7 +32,8 @@ class CacheLayout(ctypes.Structure):
 
 class Options(ctypes.Structure):
     """sconv_kv_options_t: per-head gamma stride and ring-state positions."""
-    _fields_ = [("gamma_head_stride", ctypes.c_int64), ("state_positions", ctypes.c_void_p)]
+    _fields_ = [("gamma_head_stride", ctypes.c_int64), ("state_positions", ctypes.c_void_p),
+                ("wait_timeout_ns", ctypes.c_int64), ("withhold_first_copy", ctypes.c_int64)]
 
 
 class SconvKVError(RuntimeError):
@@ -159,18 +160,22 @@ def _stream(stream):
     return int(stream)
 
 
-def _options(gamma_k, state_positions):
+def _options(gamma_k, state_positions, wait_timeout_ns=None, withhold_first_copy=False):
     """Options struct for the _ex entry points, or None for the defaults
-    (gamma [D] shared by every head, linear state).  gamma [Hkv, D] selects
-    per-head gammas; state_positions (int64 [S] on the device) a ring state."""
+    (gamma [D] shared by every head, linear state, 1 s wait limit).  gamma
+    [Hkv, D] selects per-head gammas; state_positions (int64 [S] on the
+    device) a ring state; wait_timeout_ns the kernels' wait limit."""
     per_head = gamma_k is not None and gamma_k.dim() == 2
-    if not per_head and state_positions is None:
+    if not per_head and state_positions is None and not wait_timeout_ns and \
+            not withhold_first_copy:
         return None
     if state_positions is not None and state_positions.dtype != torch.int64:
         raise TypeError("state_positions must be int64")
     o = Options()
     o.gamma_head_stride = gamma_k.shape[-1] if per_head else 0
     o.state_positions = _ptr(state_positions)
+    o.wait_timeout_ns = int(wait_timeout_ns or 0)
+    o.withhold_first_copy = 1 if withhold_first_copy else 0
     return o
 
 
@@ -191,7 +196,8 @@ def _rows(x, name):
 def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                    eps, conv_state, slot_mapping, k_cache, v_cache,
                    state_indices=None, err_flag=None, stream=None,
-                   layout=None, state_positions=None):
+                   layout=None, state_positions=None, wait_timeout_ns=None,
+                   withhold_first_copy=False):
     """Fused ShortConv K/V step over a packed varlen batch, on the GPU.
 
     k, v: bf16 [T, Hkv, D] (rows may be strided slices); cu_seqlens int32
@@ -216,7 +222,7 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
             float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
             _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_cache),
             _ptr(v_cache), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions)
+    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy)
     if opts is None:
         rc = _lib.sconv_kv_prefill_varlen(*args, _ptr(err_flag), _stream(stream))
     else:
@@ -228,7 +234,8 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
 
 def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
            slot_mapping, k_cache, v_cache, state_indices=None, err_flag=None,
-           stream=None, layout=None, state_positions=None):
+           stream=None, layout=None, state_positions=None, wait_timeout_ns=None,
+           withhold_first_copy=False):
     """Fused ShortConv K/V decode step: one new token per sequence
     (k, v: bf16 [B, Hkv, D]); same other arguments as prefill_varlen."""
     kp, rs = _rows(k, "k")
@@ -244,7 +251,7 @@ def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
             _ptr(gamma_v), float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
             _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions)
+    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy)
     if opts is None:
         rc = _lib.sconv_kv_decode(*args, _ptr(err_flag), _stream(stream))
     else:

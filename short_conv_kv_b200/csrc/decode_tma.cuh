@@ -33,6 +33,7 @@ struct DecGeom {
   int slice;      // channel groups per full slice (min(NG, 256))
   int stages;     // ring depth (sequences in flight per CTA)
   int ctas;       // CTAs along the batch
+  int withhold_first;  // testing: the first sequence's copies are never made
   int smem_ring;  // bytes of the ring
   unsigned long long timeout_ns;
 };
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
 
   // ---- producer (thread 0): sequence q (pool row si, -1 = skip) -> stage q % NS
   auto issue = [&](int q, long long si) {
+    if (q == 0 && Gm.withhold_first) return;  // nothing will complete this stage
     const int st = q % NS;
     const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
     if (si < 0) {
@@ -176,8 +178,9 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
   int issued = 0;
   auto drain = [&]() {  // after giving up: let issued loads land (bounded)
     for (int d = max(0, issued - NS); d < issued; ++d) {
+      if (d == 0 && Gm.withhold_first) continue;  // never requested
       const uint64_t t0 = global_ns();
-      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < Gm.timeout_ns) {
+      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < kDrainTimeoutNs) {
       }
     }
     bulk_wait_all();
@@ -217,11 +220,11 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
 
   for (int q = 0; q < nq; ++q) {
     const int st = q % NS;
-    if (!mbar_wait(&full[st], (q / NS) & 1, abort, Gm.timeout_ns)) {
-      if (threadIdx.x == 0) {
-        raise_flag(P.err, kFlagTimeout);
-        drain();
-      }
+    // a wait that gives up ends the whole warp at once; thread 0 first lets
+    // its issued copies land
+    if (!__all_sync(kFullMask, mbar_wait(&full[st], (q / NS) & 1, abort, Gm.timeout_ns))) {
+      if (lane == 0) raise_flag(P.err, kFlagTimeout);
+      if (threadIdx.x == 0) drain();
       return;
     }
     const bool run = s_si[q] >= 0;
@@ -278,14 +281,19 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
       if (threadIdx.x == 0 && run && W > 1) bulk_wait_read();  // write-back has read the stage
       mbar_arrive(&empty[st]);
     }
+    bool gave_up = false;
     if (threadIdx.x == 0 && q >= 1 && issued < nq) {
-      if (!mbar_wait(&empty[(q - 1) % NS], ((q - 1) / NS) & 1, abort, Gm.timeout_ns)) {
-        raise_flag(P.err, kFlagTimeout);
-        drain();
-        return;
+      if (mbar_wait(&empty[(q - 1) % NS], ((q - 1) / NS) & 1, abort, Gm.timeout_ns)) {
+        issue(issued, s_si[issued]);
+        if (++issued == nq) allow_dependent_launch();
+      } else {
+        gave_up = true;
       }
-      issue(issued, s_si[issued]);
-      if (++issued == nq) allow_dependent_launch();
+    }
+    if (__any_sync(kFullMask, gave_up)) {  // warp 0 leaves together
+      if (lane == 0) raise_flag(P.err, kFlagTimeout);
+      if (threadIdx.x == 0) drain();
+      return;
     }
   }
   // the CTA may exit once its write-backs have read shared memory; the

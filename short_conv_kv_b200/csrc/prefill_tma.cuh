@@ -94,6 +94,7 @@ struct TmaGeom {
   int slice;      // channel groups per full slice (min(NG, 256))
   int stages;     // ring depth
   int ctas;       // persistent CTAs along the token axis
+  int withhold_first;  // testing: chunk 0 is never requested (its wait runs out)
   int cut_q;      // num_tokens / ctas
   int cut_r;      // num_tokens % ctas (the first cut_r ranges take one more token)
   int cu_smem;    // cu_seqlens copied to shared memory (num_seqs < kTmaCuSmemMax)
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   const bool k_packed = kn == half && P.row_stride == P.C;
   const bool v_packed = vn == half && P.row_stride == P.C;
   auto issue = [&](int c, int st) {
+    if (c == 0 && Gm.withhold_first) return;  // nothing will complete this stage
     const int r0 = first_row + c * R;
     const int rows = min(R, tb - r0);
     mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(rows * row_bytes));
@@ -351,8 +353,9 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   // shared memory can be released (bounded as well).
   auto drain = [&]() {
     for (int d = max(0, issued - NS); d < issued; ++d) {
+      if (d == 0 && Gm.withhold_first) continue;  // never requested
       const uint64_t t0 = global_ns();
-      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < Gm.timeout_ns) {
+      while (!mbar_try_wait(&full[d % NS], (d / NS) & 1) && global_ns() - t0 < kDrainTimeoutNs) {
       }
     }
   };
@@ -535,11 +538,12 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   int s = 0;
   uint32_t ph = 0;
   for (int c = 0; c < nchunks; ++c) {
-    if (!mbar_wait(&full[s], ph, abort, Gm.timeout_ns)) {
-      if (threadIdx.x == 0) {
-        raise_flag(P.err, kFlagTimeout);
-        drain();
-      }
+    // a wait that gives up ends the whole warp at once (lanes may disagree,
+    // and no lane may be left waiting at a warp-synchronous step for one
+    // that has left); thread 0 first lets its issued copies land
+    if (!__all_sync(kFullMask, mbar_wait(&full[s], ph, abort, Gm.timeout_ns))) {
+      if (lane == 0) raise_flag(P.err, kFlagTimeout);
+      if (threadIdx.x == 0) drain();
       return;
     }
     const int r0 = first_row + c * R;
@@ -583,18 +587,23 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);  // stage fully consumed
+    bool gave_up = false;
     if (threadIdx.x == 0 && c >= 1 && issued < nchunks) {
       // refill the stage of chunk c-1 (issued == c-1+NS lands there) once
       // every warp has released it
       const int sp = s == 0 ? NS - 1 : s - 1;
       const uint32_t pp = s == 0 ? ph ^ 1u : ph;
-      if (!mbar_wait(&empty[sp], pp, abort, Gm.timeout_ns)) {
-        raise_flag(P.err, kFlagTimeout);
-        drain();
-        return;
+      if (mbar_wait(&empty[sp], pp, abort, Gm.timeout_ns)) {
+        issue(issued++, sp);
+        if (issued == nchunks) allow_dependent_launch();
+      } else {
+        gave_up = true;
       }
-      issue(issued++, sp);
-      if (issued == nchunks) allow_dependent_launch();
+    }
+    if (__any_sync(kFullMask, gave_up)) {  // warp 0 leaves together
+      if (lane == 0) raise_flag(P.err, kFlagTimeout);
+      if (threadIdx.x == 0) drain();
+      return;
     }
     if (++s == NS) {
       s = 0;

@@ -281,7 +281,10 @@ int prefill_impl(
   // + per-warp slot-offset tables + per-thread gammas
   G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes + sconv::kTmaGammaBytes;
   G.cu_smem = num_seqs < sconv::kTmaCuSmemMax ? 1 : 0;
-  G.timeout_ns = 1000000000ull;
+  G.timeout_ns = (opts && opts->wait_timeout_ns > 0)
+                     ? static_cast<unsigned long long>(opts->wait_timeout_ns)
+                     : 1000000000ull;
+  G.withhold_first = (opts && opts->withhold_first_copy) ? 1 : 0;
   const int64_t resident = static_cast<int64_t>(sm_count()) * per_sm;
   int64_t ctas = resident / ctas_y;
   const int64_t by_tokens = (num_tokens + sconv::kTmaRows - 1) / sconv::kTmaRows;
@@ -338,7 +341,10 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
   int stages = (192 * 1024 / per_sm) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
   G.smem_ring = G.stages * stage_bytes;
-  G.timeout_ns = 1000000000ull;
+  G.timeout_ns = (opts && opts->wait_timeout_ns > 0)
+                     ? static_cast<unsigned long long>(opts->wait_timeout_ns)
+                     : 1000000000ull;
+  G.withhold_first = (opts && opts->withhold_first_copy) ? 1 : 0;
   int64_t ctas = static_cast<int64_t>(sm_count()) * per_sm / ctas_y;
   const int64_t need = (static_cast<int64_t>(batch) + sconv::kDecMaxSeqs - 1) / sconv::kDecMaxSeqs;
   if (ctas < need) ctas = need;

@@ -10,6 +10,11 @@
 
 namespace sconv {
 
+// After a wait has given up, the copies already issued are still allowed to
+// land (the CTA's shared memory must outlive them): this drain is bounded
+// by its own fixed limit, whatever limit the pipeline waits were given.
+constexpr unsigned long long kDrainTimeoutNs = 1000000000ull;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
