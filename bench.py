@@ -177,6 +177,14 @@ class Workload:
                                             state="zero", page_size=64, permute_pages=True,
                                             spare_pages=64)]
             self.desc = f"W-sweep prefill T=65536, W={W}, Hkv=8, D=128, zero state, permuted pages"
+        elif name == "skew":
+            self.kind = "prefill"
+            lengths = [131072] + [16] * 1024
+            self.batches = [wl.make_prefill(lengths, Hkv=8, D=128, W=4, seed=3500 + seed_shift,
+                                            state="normal", page_size=64, permute_pages=True,
+                                            spare_pages=64)]
+            self.desc = ("skewed varlen prefill: one 131,072-token sequence + 1024 sequences of "
+                         "16 tokens, Hkv=8, D=128, W=4, N(0,1) state, permuted pages")
         elif name == "varlen":
             self.kind, self.batches = "prefill", [wl.varlen(seed=3000 + seed_shift)]
             self.desc = "varlen prefill 32 seqs U[512,8192], Hkv=8, D=128, W=4, N(0,1) state, permuted pages"
@@ -702,7 +710,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="single",
-                    choices=["single", "varlen", "decode", "decode_ring", "long", "wsweep2",
+                    choices=["single", "varlen", "skew", "decode", "decode_ring", "long", "wsweep2",
                              "wsweep4", "wsweep8",
                              "single_mx", "varlen_mx", "decode_mx", "long_mx", "wsweep2_mx",
                              "wsweep4_mx", "wsweep8_mx"])

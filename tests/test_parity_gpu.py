@@ -413,3 +413,12 @@ def test_deterministic():
     r2 = gu.run_gpu_prefill(b)
     for x, y in zip(r1, r2):
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+def test_skewed_lengths_full():
+    """One long sequence among many short ones (the even token split puts
+    many CTAs inside the long one and several short sequences in one CTA)."""
+    lengths = [4000] + [3, 16, 1, 0, 7] * 60
+    b = wl.make_prefill(lengths, Hkv=4, D=128, W=4, seed=905, state="normal",
+                        page_size=16, spare_pages=4)
+    gu.full_parity(b)
