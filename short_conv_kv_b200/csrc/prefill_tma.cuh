@@ -2,8 +2,10 @@
 // (sm_100a).
 //
 // Work split.  The packed token axis [0, T) is cut into `ctas` contiguous
-// ranges of near-equal length, one per persistent CTA (x), and the channel
-// groups into slices of at most 256 groups of 8 channels (y).  A cut that
+// ranges of near-equal cost (a token costs 1, a sequence start a fixed
+// number of tokens; one sequence is cut evenly), one per persistent CTA
+// (x), and the channel groups into slices of at most 256 groups of 8
+// channels (y).  A cut that
 // would fall on positions 1..W-2 of a sequence is moved to position W-1 (or
 // to the sequence's end), so the CTA holding position 0 of a sequence also
 // holds every position whose window reaches into the old conv_state: that
@@ -95,6 +97,7 @@ struct TmaGeom {
   int stages;     // ring depth
   int ctas;       // persistent CTAs along the token axis
   int withhold_first;  // testing: chunk 0 is never requested (its wait runs out)
+  int seq_cost;   // weight of a sequence start, in tokens (cut by cost)
   int cut_q;      // num_tokens / ctas
   int cut_r;      // num_tokens % ctas (the first cut_r ranges take one more token)
   int cu_smem;    // cu_seqlens copied to shared memory (num_seqs < kTmaCuSmemMax)
@@ -220,8 +223,8 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   // first_row + c*R ... whatever the final start is; rows in front of the
   // final start are skipped by the consumers.
   auto cut_even = [&](int b) -> int { return min(b * Gm.cut_q + min(b, Gm.cut_r), T); };
-  const int first_row = cut_even(blockIdx.x);
-  int tb = cut_even(blockIdx.x + 1);  // end of the range (final value set below)
+  int first_row = cut_even(blockIdx.x);  // (final value set below)
+  int tb = cut_even(blockIdx.x + 1);      // end of the range (final value set below)
 
   // =================================================================== producer
   // Issue chunk c into stage `st` (= c % NS, tracked by the caller).
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     // full chunks that lie inside the even range: requested at once (block
     // layout only; in the W=4 bf16 instance the extra live values spill at
     // its 128-register cap, so it requests after the cut)
-    const int spec = min(NS, (tb - first_row) / R);
+    const int spec = S == 1 ? min(NS, (tb - first_row) / R) : 0;
     for (; issued < spec; ++issued) issue(issued, issued);
   }
   if (Gm.cu_smem)
@@ -303,9 +306,27 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     return lo;
   };
   // start of range b: even cut, moved off positions 1..W-2 of a sequence
+  // Cut by cost: a token weighs 1 and a sequence start Gm.seq_cost tokens
+  // (its state read and write are latency the CTA cannot hide), so CTAs
+  // full of short sequences get fewer tokens.  Sequence i's start sits at
+  // weight cu[i] + cost*i; target weight X falls in the last sequence whose
+  // start is at or below it.  A single sequence keeps the even split.
+  auto base_cut = [&](int b) -> int {
+    if (S <= 1 || Gm.seq_cost == 0) return cut_even(b);
+    const long long cost = Gm.seq_cost;
+    const long long X = static_cast<long long>(b) * (T + cost * S) / Gm.ctas;
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu(mid) + cost * mid <= X) lo = mid; else hi = mid - 1;
+    }
+    long long t = cu(lo) + max(0ll, X - (cu(lo) + cost * lo) - cost);
+    t = min(t, static_cast<long long>(cu(lo + 1)));
+    return static_cast<int>(min(max(t, 0ll), static_cast<long long>(T)));
+  };
   static_assert(R > W - 2, "a moved cut must stay inside the first chunk");
   auto cut = [&](int b) -> int {
-    const int s0 = cut_even(b);
+    const int s0 = base_cut(b);
     if (s0 >= T) return T;
     int s = s0;
     if (W > 1) {
@@ -326,6 +347,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     for (int i = threadIdx.x; i < S && ok; i += blockDim.x) ok = cu(i) <= cu(i + 1);
     if (!ok) raise_flag(P.err, kFlagCuSeqlens);
   }
+  first_row = base_cut(blockIdx.x);  // equals the even cut for a single sequence
   const int ta = cut(blockIdx.x);
   // rows of chunk 0 in front of ta, one copy per warp in shared memory (read
   // once per 32-row window: a register here spills in the W=4 bf16 instance)

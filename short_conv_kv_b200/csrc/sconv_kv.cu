@@ -291,6 +291,10 @@ int prefill_impl(
   if (ctas > by_tokens) ctas = by_tokens;
   if (ctas < 1) ctas = 1;
   G.ctas = static_cast<int>(ctas);
+#ifndef SCONV_PREFILL_SEQ_COST
+#define SCONV_PREFILL_SEQ_COST 16  // tokens a sequence start is worth when cutting ranges
+#endif
+  G.seq_cost = SCONV_PREFILL_SEQ_COST;
   G.cut_q = static_cast<int>(num_tokens / ctas);
   G.cut_r = static_cast<int>(num_tokens % ctas);
   const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 48 +
