@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "sconv_kv.h"
 #include "common.cuh"
 #include "decode_tma.cuh"
@@ -89,11 +91,16 @@ DecFn pick_decode(int W, int D, bool mx, bool lv) {
             : Pick<DecFn, DecodeKs<false, false>::K>::get(W, D);
 }
 
+// Host-side caches (SM counts, shared-memory attributes, scratch addresses)
+// are shared by every host thread that calls the library.
+std::mutex g_cache_mutex;
+
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  std::lock_guard<std::mutex> lock(g_cache_mutex);
   if (dev < 64 && cached[dev] > 0) return cached[dev];
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
@@ -105,23 +112,32 @@ int sm_count() {
 // Opt a kernel into `bytes` of dynamic shared memory (once per kernel and
 // size; host-side attribute, not a stream operation).
 bool smem_attr_set(const void* fn, size_t bytes) {
-  static const void* done_fn[256];
-  static size_t done_bytes[256];
+  static const void* done_fn[512];
+  static int done_dev[512];
+  static size_t done_bytes[512];
   static int n_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(g_cache_mutex);
+  // the attribute belongs to the function in one device's context
   for (int i = 0; i < n_done; ++i)
-    if (done_fn[i] == fn && done_bytes[i] >= bytes) return true;
+    if (done_fn[i] == fn && done_dev[i] == dev && done_bytes[i] >= bytes) return true;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(bytes)) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
   for (int i = 0; i < n_done; ++i)
-    if (done_fn[i] == fn) {
+    if (done_fn[i] == fn && done_dev[i] == dev) {
       done_bytes[i] = bytes;
       return true;
     }
-  if (n_done < 256) {
+  if (n_done < 512) {
     done_fn[n_done] = fn;
+    done_dev[n_done] = dev;
     done_bytes[n_done] = bytes;
     ++n_done;
   }
@@ -446,6 +462,7 @@ unsigned char* noalloc_scratch() {
   static unsigned char* cached[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_cache_mutex);
   if (!cached[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
