@@ -41,8 +41,15 @@ from short_conv_kv_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-KERNEL_SOURCES = [os.path.join(ROOT, "short_conv_kv_b200", "csrc", f)
-                  for f in ("common.cuh", "tma.cuh", "prefill_tma.cuh", "decode_tma.cuh", "sconv_kv.cu")]
+# Sources each kernel is built from (device code and its host-side launch
+# geometry); a committed profile counts only while these are unchanged.
+_CSRC = os.path.join(ROOT, "short_conv_kv_b200", "csrc")
+KERNEL_SOURCES = {
+    "prefill_tma_kernel": [os.path.join(_CSRC, f) for f in
+                           ("common.cuh", "tma.cuh", "prefill_tma.cuh", "sconv_kv.cu")],
+    "decode_tma_kernel": [os.path.join(_CSRC, f) for f in
+                          ("common.cuh", "tma.cuh", "decode_tma.cuh", "sconv_kv.cu")],
+}
 
 
 # ------------------------------------------------------------------ helpers
@@ -63,9 +70,10 @@ def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8, mx=False, ring=Fals
     return tokens * per_token + seqs * per_seq + per_launch
 
 
-def source_hash():
+def source_hash(kernel):
+    """Hash of the sources of `kernel` (a key of KERNEL_SOURCES)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -90,7 +98,8 @@ def profile_traffic(kernel_tag):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha256") != source_hash():
+    kernel = "decode_tma_kernel" if kernel_tag.startswith("decode") else "prefill_tma_kernel"
+    if vals.get("source_sha256") != source_hash(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full"])
