@@ -88,12 +88,18 @@ __device__ __forceinline__ void allow_dependent_launch() {
 
 // One bulk copy global -> this CTA's shared memory, completion signalled on
 // `bar` as transaction bytes.  dst, src 16-byte aligned; bytes % 16 == 0.
-// (Plain load: no cluster multicast.)
+// (Plain load: no cluster multicast.)  The copy carries an L2 evict-first
+// policy: the kernels read every input row exactly once, so the next reads
+// should replace these lines rather than the cache rows just written
+// (measured on B200: 8192-token prefill 18.4 -> 17.0 us, ring-state decode
+// 7.7 -> 7.0 us; launches larger than L2 about 1 % slower).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
+      "{\n\t.reg .b64 pol;\n\t"
+      "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], pol;\n\t}" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
