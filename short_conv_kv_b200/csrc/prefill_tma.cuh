@@ -582,14 +582,33 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     const unsigned char* stage = my_ring + static_cast<size_t>(s) * R * row_bytes;
     if (next >= r0 + rows && !skip) {
       // fast path: up to R tokens of one sequence, no branches (rows past
-      // the end of the range compute on stale data and are not stored)
+      // the end of the range compute on stale data and are not stored).
+      // Where the unroll is shorter than a chunk, the tokens go in groups of
+      // UF and a range's last, partial chunk skips the groups wholly past
+      // its end (a short launch's ranges end in such a chunk).
+      constexpr int UF = fast_unroll<W, MX>();
+      if constexpr (UF < R) {
+        static_assert(R % UF == 0, "a chunk is a whole number of groups");
+        for (int rb = 0; rb < rows; rb += UF) {
+#pragma unroll
+          for (int u = 0; u < UF; ++u) {
+            const int r = rb + u;
+            const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
+            float2 acc[4];
+            conv_step<W>(tw, win, xr, acc);
+            const long long off = warp_off[sbase + r];
+            NORM_STORE(active && r < rows && off >= 0);
+          }
+        }
+      } else {
 #pragma unroll fast_unroll<W, MX>()
-      for (int r = 0; r < R; ++r) {
-        const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
-        float2 acc[4];
-        conv_step<W>(tw, win, xr, acc);
-        const long long off = warp_off[sbase + r];
-        NORM_STORE(active && r < rows && off >= 0);
+        for (int r = 0; r < R; ++r) {
+          const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
+          float2 acc[4];
+          conv_step<W>(tw, win, xr, acc);
+          const long long off = warp_off[sbase + r];
+          NORM_STORE(active && r < rows && off >= 0);
+        }
       }
     } else {
       for (int r = 0; r < rows; ++r) {
