@@ -34,6 +34,16 @@ def test_mx_single_8192():
     gu.full_parity_mx(wl.single())
 
 
+@pytest.mark.parametrize("i", range(7))
+def test_mx_partial_last_chunks(i):
+    """MXFP8 store (2-token groups) over ranges ending in a partial chunk of
+    every length 1..7."""
+    from tests.test_parity_gpu import tail_lengths
+    T = tail_lengths()[i]
+    gu.full_parity_mx(wl.make_prefill([T], Hkv=8, D=128, W=4, seed=2200 + i, state="normal",
+                                      page_size=64, permute_pages=True))
+
+
 @pytest.mark.parametrize("W", [1, 2, 4, 8])
 def test_mx_every_w(W):
     b = wl.make_prefill([300, 1, 0, 77, 2], Hkv=4, D=128, W=W, seed=1600 + W,

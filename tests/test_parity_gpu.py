@@ -26,6 +26,15 @@ def _binding():
     return binding
 
 
+def tail_lengths():
+    """Single-sequence lengths that give every persistent CTA of the W <= 4
+    prefill (two per SM, 8-row chunks) exactly k rows, k = 25..31: ranges
+    ending in partial chunks of 1..7 rows, whose unrolled groups wholly
+    past the end are skipped."""
+    ctas = 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    return [ctas * k for k in range(25, 32)]
+
+
 # ----------------------------------------------------------- named configs
 
 def test_tiny_full():
@@ -36,6 +45,15 @@ def test_tiny_full():
 def test_single_8192_full():
     """One 8192-token sequence, Hkv=8, D=128, W=4, contiguous cache."""
     gu.full_parity(wl.single())
+
+
+@pytest.mark.parametrize("i", range(7))
+def test_partial_last_chunks_full(i):
+    """Ranges ending in a partial chunk of every length 1..7 (one sequence,
+    W=4, N(0,1) state, permuted pages)."""
+    T = tail_lengths()[i]
+    gu.full_parity(wl.make_prefill([T], Hkv=8, D=128, W=4, seed=2100 + i, state="normal",
+                                   page_size=64, permute_pages=True))
 
 
 def _sample_tokens(cu, W, rng, n_random=2000, tile=32):
