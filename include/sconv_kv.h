@@ -39,6 +39,11 @@
  *     SCONV_KV_FLAG_* bit is OR-ed into *err_flag (if err_flag is not NULL);
  *     the caller clears *err_flag and reads it after synchronising.
  *
+ * Cache behaviour: the fused kernels read each k/v row (and, in decode,
+ * each old conv_state row) exactly once and load them with an L2
+ * evict-first policy, so later kernels find the cache rows just written
+ * in L2 rather than these inputs.
+ *
  * Preconditions the library cannot check without synchronising (results are
  * unspecified when they are violated): non-negative slots are unique within
  * a call; state indices are unique within a call; k/v do not alias the
