@@ -34,6 +34,10 @@ MUTANTS = [
     ("e4m3_overflow_nan", "if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 448.0) return (uint8_t)(sign | 0x7F);"),
     ("e4m3_truncates", "double r = ldexp(rint(ldexp(a, -q)), q);", "double r = ldexp(floor(ldexp(a, -q)), q);"),
     ("e4m3_subnormal_grid", "if (q < -9) q = -9;", "if (q < -10) q = -10;"),
+    ("eps_dropped", "1.0 / sqrt(ss / (double)D + eps)", "1.0 / sqrt(ss / (double)D)"),
+    ("gamma_in_sum_of_squares", "ss += yh[d] * yh[d];",
+     "ss += yh[d] * yh[d] * (double)gh[d] * (double)gh[d];"),
+    ("state_indices_ignored", "state_indices ? state_indices[i] : i", "i"),
 ]
 
 
