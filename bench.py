@@ -2,18 +2,28 @@
 """Benchmark of the fused ShortConv K/V step (tokens/s and achieved HBM GB/s).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload single|varlen|decode|long|wsweep2|wsweep8]
+                    [--workload long|single|varlen|decode|...] [--no-configs]
 
 One step = one pass of the whole step (window assembly + causal conv, RMSNorm,
-bf16 scatter into the paged cache, conv_state update) over one batch,
-through the C ABI.  Default workload: one 8192-token sequence, Hkv=8, D=128,
-W=4, zero state, contiguous cache (page_size 64).
+bf16 scatter into the paged cache, conv_state update) over one batch of
+synthetic input, through the C ABI.  Default workload (the headline line):
+the long-context chunked prefill -- one 1,048,576-token sequence, Hkv=8,
+D=128, W=4, processed as 16 calls of 65,536 tokens with the conv_state
+carried from call to call, paged cache (page 64, seeded page permutation).
+A step of that workload is the whole sequence, i.e. 16 kernel launches.
 
 Timing: W warm-up steps, then exactly K steps captured in one CUDA graph and
 replayed once, bracketed by a barrier + synchronize on both sides and by CUDA
-events on the replay stream; time / K is both the step time and the kernel's
-average launch duration (one launch per step); max over ranks.
-Inputs rotate over enough buffer sets that each step's bytes exceed L2.
+events on the replay stream; a sleep kernel queued in front of the start
+event keeps the GPU busy while the host submits the graph, so the region
+holds the launches only.  time / (K x launches per step) is the kernel's
+average launch duration; max over ranks.  Inputs rotate over enough buffer
+sets that each step's bytes exceed L2.
+
+The `configs` key of the line times the other full-size workloads the same
+way (8192-token single prefill, 32-sequence varlen batch, 1024-sequence
+decode step, W=2 and W=8 65,536-token launches), each over enough launches
+for a region of at least ~20 ms.
 
 Under torchrun each rank runs its own independent batch (the step shards by
 sequence with no exchange: weak scaling); rank 0 prints one JSON line.
@@ -40,6 +50,9 @@ if ROOT not in sys.path:
 from short_conv_kv_b200 import workloads as wl  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+# A sleep kernel of about 2 ms at the B200's SM clock, queued ahead of each
+# timed region (outside it) while the host submits the graph.
+SLEEP_CYCLES = 4_000_000
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 # Sources each kernel is built from (device code and its host-side launch
 # geometry); a committed profile counts only while these are unchanged.
@@ -168,13 +181,18 @@ class ClockSampler:
 # ------------------------------------------------------------------ workloads
 
 class Workload:
-    """Device-resident rotating input sets plus host copies for e2e."""
+    """Device-resident rotating input sets plus host copies for e2e.
+
+    A step is `launches_per_step` calls (16 chunk calls for the long-context
+    workload, one call otherwise); every launch of a workload moves the
+    same algorithmic bytes (`bytes_per_launch`)."""
 
     def __init__(self, name, rank):
         self.mx = name.endswith("_mx")  # MXFP8 cache store variant
         name = name[:-3] if self.mx else name
         self.ring = name.endswith("_ring")  # ring-buffer conv_state (decode)
         self.name, self.rank = name, rank
+        self.launches_per_step = 1
         seed_shift = 97 * rank
         if name == "single":
             self.kind, self.batches = "prefill", [wl.single(seed=2000 + seed_shift)]
@@ -194,13 +212,25 @@ class Workload:
                                             spare_pages=64)]
             self.desc = ("skewed varlen prefill: one 131,072-token sequence + 1024 sequences of "
                          "16 tokens, Hkv=8, D=128, W=4, N(0,1) state, permuted pages")
+        elif name == "many":
+            self.kind = "prefill"
+            g = torch.Generator().manual_seed(3600 + seed_shift)
+            lengths = torch.randint(32, 97, (1900,), generator=g).tolist()
+            self.batches = [wl.make_prefill(lengths, Hkv=8, D=128, W=4, seed=3601 + seed_shift,
+                                            state="normal", page_size=64, permute_pages=True,
+                                            spare_pages=64)]
+            self.desc = ("many-sequence varlen prefill: 1900 sequences of 32..96 tokens, "
+                         "Hkv=8, D=128, W=4, N(0,1) state, permuted pages")
         elif name == "varlen":
             self.kind, self.batches = "prefill", [wl.varlen(seed=3000 + seed_shift)]
             self.desc = "varlen prefill 32 seqs U[512,8192], Hkv=8, D=128, W=4, N(0,1) state, permuted pages"
         elif name == "long":
             self.kind = "long"
             self.long = wl.long_context(seed=5000 + seed_shift)
-            self.desc = "long-context chunked prefill 1,048,576 tokens in 65,536-token chunks, W=4, state carried"
+            self.launches_per_step = self.long.num_chunks
+            self.desc = ("long-context chunked prefill: one 1,048,576-token sequence as 16 calls "
+                         "of 65,536 tokens, state carried, Hkv=8, D=128, W=4, zero initial "
+                         "state, paged cache (page 64, seeded permutation)")
         elif name in ("decode", "decode_ring"):
             self.kind = "decode"
             self.dec = wl.decode(seed=4000 + seed_shift)
@@ -218,12 +248,12 @@ class Workload:
         if self.kind == "prefill":
             b = self.batches[0]
             self.W, self.Hkv, self.D = b.W, b.Hkv, b.D
-            self.tokens_per_step, self.seqs_per_step = b.num_tokens, b.num_seqs
-            self.bytes_per_step = algorithmic_bytes(b.num_tokens, b.num_seqs, b.W, b.Hkv, b.D,
-                                                    mx=self.mx)
+            self.tokens_per_launch, self.seqs_per_step = b.num_tokens, b.num_seqs
+            self.bytes_per_launch = algorithmic_bytes(b.num_tokens, b.num_seqs, b.W, b.Hkv, b.D,
+                                                      mx=self.mx)
             shared = dict(conv_w_k=b.conv_w_k.to(dev), conv_w_v=b.conv_w_v.to(dev),
                           gamma_k=b.gamma_k.to(dev), gamma_v=b.gamma_v.to(dev))
-            R = max(1, math.ceil(3 * L2_BYTES / self.bytes_per_step))
+            R = max(1, math.ceil(3 * L2_BYTES / self.bytes_per_launch))
             self.rotation = R
             for r in range(R):
                 self.calls_args.append(dict(
@@ -234,8 +264,8 @@ class Workload:
         elif self.kind == "long":
             s = self.long
             self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
-            self.tokens_per_step, self.seqs_per_step = s.chunk, 1
-            self.bytes_per_step = algorithmic_bytes(s.chunk, 1, s.W, s.Hkv, s.D, mx=self.mx)
+            self.tokens_per_launch, self.seqs_per_step = s.chunk, 1
+            self.bytes_per_launch = algorithmic_bytes(s.chunk, 1, s.W, s.Hkv, s.D, mx=self.mx)
             shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
                           gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
                           conv_state=s.initial_state().to(dev),
@@ -248,13 +278,13 @@ class Workload:
         else:
             s = self.dec
             self.W, self.Hkv, self.D = s.W, s.Hkv, s.D
-            self.tokens_per_step, self.seqs_per_step = s.batch, s.batch
-            self.bytes_per_step = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D, mx=self.mx,
-                                                    ring=self.ring)
+            self.tokens_per_launch, self.seqs_per_step = s.batch, s.batch
+            self.bytes_per_launch = algorithmic_bytes(s.batch, s.batch, s.W, s.Hkv, s.D,
+                                                      mx=self.mx, ring=self.ring)
             shared = dict(conv_w_k=s.conv_w_k.to(dev), conv_w_v=s.conv_w_v.to(dev),
                           gamma_k=s.gamma_k.to(dev), gamma_v=s.gamma_v.to(dev), eps=s.eps,
                           k_cache=s.empty_cache().to(dev), v_cache=s.empty_cache().to(dev))
-            R = max(2, math.ceil(3 * L2_BYTES / self.bytes_per_step))
+            R = max(2, math.ceil(3 * L2_BYTES / self.bytes_per_launch))
             self.rotation = R
             states = [s.conv_state.to(dev) for _ in range(min(R, 16))]
             for r in range(R):
@@ -265,6 +295,8 @@ class Workload:
                     pos = s.start_len.astype(np.int64) + (r % 64)
                     a["state_positions"] = torch.from_numpy(pos).to(dev)
                 self.calls_args.append(a)
+        self.tokens_per_step = self.tokens_per_launch * self.launches_per_step
+        self.bytes_per_step = self.bytes_per_launch * self.launches_per_step
 
         if self.mx:
             # MXFP8 store: uint8 E4M3 data + E8M0 scale caches in place of
@@ -311,25 +343,25 @@ class Workload:
 
 # ------------------------------------------------------------------ unfused chain
 
-def time_unfused(work, K, Wu, dev):
+def time_unfused(work, n, Wu, dev):
     """The same step as the library's four unfused stage kernels (conv ->
     y, rmsnorm -> z, scatter, state update; bf16 intermediates in HBM) over
-    the same rotating buffers, K steps in one CUDA graph replay (the fused
-    kernel's timing method).  Context for the fused-versus-unfused claim
-    ("SGLang and Miles announce day-0 Inkling support", aib.vote English
-    news item, paragraph 2)."""
+    the same rotating buffers, n calls in one CUDA graph replay (the fused
+    kernel's timing method); returns ms per call.  Context for the
+    fused-versus-unfused claim ("SGLang and Miles announce day-0 Inkling
+    support", aib.vote English news item, paragraph 2)."""
     from short_conv_kv_b200 import binding
     stream = torch.cuda.Stream(device=dev)
-    T = work.tokens_per_step
+    T = work.tokens_per_launch
     C = work.Hkv * work.D
     y = torch.empty(T, 2 * C, dtype=torch.bfloat16, device=dev)
     z = torch.empty_like(y)
-    n = len(work.calls_args)
+    m = len(work.calls_args)
     if work.kind == "decode":
         cu = torch.arange(T + 1, dtype=torch.int32, device=dev)
 
     def chain(i, s):
-        a = work.calls_args[i % n]
+        a = work.calls_args[i % m]
         return binding.prepare_unfused(
             a["k"], a["v"], a["cu_seqlens"] if work.kind != "decode" else cu, a["conv_w_k"],
             a["conv_w_v"], a["gamma_k"], a["gamma_v"], a["eps"], a["conv_state"],
@@ -342,19 +374,21 @@ def time_unfused(work, K, Wu, dev):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         cap = torch.cuda.current_stream()
-        runs = [chain(i, cap) for i in range(K)]
+        runs = [chain(i, cap) for i in range(n)]
         for r in runs:
             r()
     g.replay()
     torch.cuda.synchronize()
     s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(SLEEP_CYCLES)  # (current stream) the host submits meanwhile
+    stream.wait_stream(torch.cuda.current_stream())
     s_ev.record(stream)
     with torch.cuda.stream(stream):
         g.replay()
     e_ev.record(stream)
     e_ev.synchronize()
     del g
-    return s_ev.elapsed_time(e_ev) / K
+    return s_ev.elapsed_time(e_ev) / n
 
 
 # ------------------------------------------------------------------ our arm
@@ -389,23 +423,28 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
-def time_graph(work, K, Wu, dev, world, local):
-    """Warm-up W eager steps, then K steps captured in one CUDA graph (kernel
-    nodes back to back, nothing between them) and replayed once as the timed
-    region.  The kernel's average launch duration is the region's time / K
-    (so it includes the short gaps between consecutive launches)."""
+def time_graph(work, K, Wu, dev, world, local, profile_range=False):
+    """Warm-up W eager steps, then K steps (K x launches_per_step calls)
+    captured in one CUDA graph (kernel nodes back to back, nothing between
+    them) and replayed once as the timed region.  A sleep kernel queued in
+    front of the start event keeps the GPU busy while the host submits the
+    replay, so the region holds the launches (and the short gaps between
+    consecutive launches) only.  With profile_range the timed replay is
+    bracketed by cudaProfilerStart/Stop, for a profiler that captures the
+    whole replay as one range."""
+    lps = work.launches_per_step
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
-        for i in range(Wu):
+        for i in range(Wu * lps):
             work.prepared(i, stream)()
     stream.synchronize()
 
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         cap = torch.cuda.current_stream()
-        calls = [work.prepared(i, cap) for i in range(K)]
-        for i in range(K):
-            calls[i]()
+        calls = [work.prepared(i, cap) for i in range(K * lps)]
+        for c in calls:
+            c()
     # one untimed replay uploads the graph and warms it
     g.replay()
     torch.cuda.synchronize()
@@ -415,11 +454,17 @@ def time_graph(work, K, Wu, dev, world, local):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(SLEEP_CYCLES)
+        if profile_range:
+            torch.cuda.profiler.start()
         outer_s.record(stream)
         with torch.cuda.stream(stream):
             g.replay()
         outer_e.record(stream)
         outer_e.synchronize()
+        if profile_range:
+            torch.cuda.profiler.stop()
     torch.cuda.synchronize()
     barrier(world)
     total_ms = outer_s.elapsed_time(outer_e)
@@ -569,40 +614,118 @@ def cpu_oracle_baseline(work, budget_s=12.0):
                       f"host has {os.cpu_count()} cores)"}
 
 
+# Workloads timed beside the headline line (the other full-size
+# configurations): name -> label of the `configs` entry.
+SIDE_CONFIGS = [
+    ("single", "single-sequence prefill T=8192"),
+    ("varlen", "varlen prefill, 32 sequences"),
+    ("decode", "decode step, 1024 sequences"),
+    ("wsweep2", "65,536-token prefill, W=2"),
+    ("wsweep8", "65,536-token prefill, W=8"),
+]
+SIDE_MIN_MS = 20.0     # timed region per side workload, at least
+SIDE_MAX_LAUNCHES = 2500
+
+
+def line_roofline(work, kern_ms, peaks, peak_src, traffic):
+    achieved = work.bytes_per_launch / (kern_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)",
+            "frac_of_8tbs": achieved / 8000.0,
+            "algorithmic_bytes_per_launch": work.bytes_per_launch,
+            "kernel_ms_per_launch": kern_ms}
+
+
+def time_side_config(name, label, K, Wu, dev, world, local, peaks, peak_src):
+    """One full-size side workload timed like the headline (graph replay,
+    rotating buffers), over max(K, enough launches for SIDE_MIN_MS) launches."""
+    work = Workload(name, 0)
+    work.setup(dev)
+    # a short eager probe sets the number of launches of the timed region
+    stream = torch.cuda.Stream(device=dev)
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            work.prepared(i, stream)()
+        s_ev.record(stream)
+        for i in range(10):
+            work.prepared(i, stream)()
+        e_ev.record(stream)
+    e_ev.synchronize()
+    est = max(s_ev.elapsed_time(e_ev) / 10, 1e-3)
+    n = int(min(SIDE_MAX_LAUNCHES, max(K, math.ceil(SIDE_MIN_MS / est))))
+    total_ms, clocks = time_graph(work, n, Wu, dev, world, local)
+    total_ms = max_over_ranks(total_ms, world)
+    kern_ms = total_ms / n
+    r = line_roofline(work, kern_ms, peaks, peak_src,
+                      profile_traffic(f"{work.kernel_tag()}_{name}"))
+    out = {"label": label, "workload": work.desc, "launches": n,
+           "ms_per_launch": kern_ms, "tokens_per_s": world * work.tokens_per_launch / (kern_ms / 1e3),
+           "algorithmic_bytes_per_launch": work.bytes_per_launch,
+           "achieved_gbs": r["achieved"], "frac": r["frac"], "frac_of_8tbs": r["frac_of_8tbs"],
+           "traffic": r["traffic"], "clocks": clocks}
+    del work
+    torch.cuda.empty_cache()
+    return out, n
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
     work = Workload(args.workload, rank)
     work.setup(dev)
     K, Wu = args.steps, args.warmup
-    total_ms, clocks = time_graph(work, K, Wu, dev, world, local)
+    lps = work.launches_per_step
+    total_ms, clocks = time_graph(work, K, Wu, dev, world, local,
+                                  profile_range=args.profile_range)
     total_ms = max_over_ranks(total_ms, world)
+    if args.profile_range:
+        # the profiled run only needs its timed region; nothing else runs
+        if rank == 0:
+            print(json.dumps({"profile_range": work.desc, "steps": K,
+                              "launches": K * lps, "ms": total_ms}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     ms_per_step = total_ms / K
-    kern_ms = ms_per_step  # one launch per step
+    kern_ms = total_ms / (K * lps)  # average launch duration
     value = world * work.tokens_per_step * K / (total_ms / 1e3)
+    launches = K * lps
     e2e = None
     if not work.mx:  # the end-to-end leg is measured on the bf16 store
         e2e_ms, h2d, d2h = time_e2e(work, args.e2e_steps, dev)
         e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": world * work.tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": world * work.tokens_per_launch / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "method": "pinned host buffers; upload of the inputs, the step, and download "
-                         "of the written cache rows + new state, pipelined over two buffer "
-                         "sets on three streams"}
+               "method": ("pinned host buffers; per call: upload of the inputs, the step, and "
+                          "download of the written cache rows + new state, pipelined over two "
+                          "buffer sets on three streams" +
+                          ("; a step here is one 65,536-token call of the chunked sequence "
+                           "(state carried from call to call)" if work.kind == "long" else ""))}
     unfused = None
     if not work.mx and not work.ring and not args.no_unfused:
-        Ku = min(K, 50)
+        Ku = min(launches, 50)
         un_ms = max_over_ranks(time_unfused(work, Ku, Wu, dev), world)
-        T, C = work.tokens_per_step, work.Hkv * work.D
-        un_bytes = work.bytes_per_step + T * 2 * C * 2 * 4  # + y and z, each written and read
-        unfused = {"ms_per_step": un_ms, "steps": Ku, "fused_speedup": un_ms / ms_per_step,
-                   "algorithmic_bytes_per_step": un_bytes,
+        T, C = work.tokens_per_launch, work.Hkv * work.D
+        un_bytes = work.bytes_per_launch + T * 2 * C * 2 * 4  # + y and z, each written and read
+        unfused = {"ms_per_launch": un_ms, "launches": Ku, "fused_speedup": un_ms / kern_ms,
+                   "algorithmic_bytes_per_launch": un_bytes,
                    "achieved_gbs": un_bytes / (un_ms / 1e3) / 1e9,
                    "kind": "the library's unfused stage kernels: conv -> y, rmsnorm -> z, "
                            "scatter, state update (4 launches, bf16 intermediates in HBM), "
                            "one CUDA graph replay"}
     peaks, peak_src = measured_peaks()
-    achieved = work.bytes_per_step / (kern_ms / 1e3) / 1e9
+    configs = None
+    side_launches = 0
+    if not args.no_configs and args.workload == "long":
+        configs = {}
+        del work.calls_args  # free the headline's buffers first
+        torch.cuda.empty_cache()
+        for name, label in SIDE_CONFIGS:
+            configs[name], n = time_side_config(name, label, K, Wu, dev, world, local, peaks,
+                                                peak_src)
+            side_launches += n
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_baseline(work)
@@ -616,23 +739,22 @@ def run_ours(args):
                        "storage": ("bf16 in, MXFP8 cache, bf16 state, fp32 math" if work.mx
                                    else "bf16 in, bf16 cache/state, fp32 math"),
                        "tokens_per_step_per_gpu": work.tokens_per_step,
+                       "launches_per_step": lps,
+                       "tokens_per_launch": work.tokens_per_launch,
                        "seqs_per_step_per_gpu": work.seqs_per_step, "W": work.W,
                        "num_kv_heads": work.Hkv, "head_dim": work.D,
                        "parallelism": f"{world} independent replicas (sequence sharding, no collective)",
                        "l2": f"inputs rotate over {work.rotation} buffer sets "
-                             f"({work.rotation * work.bytes_per_step / 1e6:.0f} MB) > L2",
+                             f"({work.rotation * work.bytes_per_launch / 1e6:.0f} MB) > L2",
                        "timing": "K steps in one CUDA graph replay, CUDA events around the replay"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": profile_traffic(f"{work.kernel_tag()}_{args.workload}"),
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)",
-                         "frac_of_8tbs": achieved / 8000.0,
-                         "algorithmic_bytes_per_launch": work.bytes_per_step,
-                         "kernel_ms_per_launch": kern_ms},
+            "roofline": line_roofline(work, kern_ms, peaks, peak_src,
+                                      profile_traffic(f"{work.kernel_tag()}_{args.workload}")),
+            "configs": configs,
             "cpu_baseline": cpu,
             "unfused_chain": unfused,
             "e2e": e2e,
-            "gpu_launches": K,
+            "gpu_launches": launches,
+            "gpu_launches_side_configs": side_launches,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -715,18 +837,23 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="single",
-                    choices=["single", "varlen", "skew", "decode", "decode_ring", "long", "wsweep2",
-                             "wsweep4", "wsweep8",
+    ap.add_argument("--workload", default="long",
+                    choices=["long", "single", "varlen", "skew", "decode", "decode_ring", "wsweep2",
+                             "wsweep4", "wsweep8", "many",
                              "single_mx", "varlen_mx", "decode_mx", "long_mx", "wsweep2_mx",
                              "wsweep4_mx", "wsweep8_mx"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true",
                     help="skip timing the unfused four-kernel chain (context only)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the side workloads of the `configs` key")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket the timed replay with cudaProfilerStart/Stop and run nothing "
+                         "else (for a range capture of the DRAM counters)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

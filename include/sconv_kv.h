@@ -342,7 +342,12 @@ SCONV_KV_API int sconv_kv_decode_mxfp8_ex(
  *   gamma[d] per (token, head), rounded to bf16.
  * sconv_kv_stage_scatter: cache[slot_mapping[t]] = z[t] (K half into
  *   k_cache, V half into v_cache); slot < 0 skips the token; a slot past
- *   the cache is skipped and flagged.
+ *   the cache is skipped and flagged.  cu_seqlens (with num_seqs >= 1, W
+ *   and the state pool as given to the other stages) is optional: when it
+ *   is not NULL, the tokens of a sequence that the other stages skip (a
+ *   malformed cu_seqlens entry, or for W > 1 a state index outside the
+ *   pool) are not written either, so the chain leaves the same cache slots
+ *   untouched as the fused step; when it is NULL every token is written.
  * sconv_kv_stage_state_update: each sequence's state = the last W-1 raw
  *   rows of (old state ++ its rows), in place; must run after every reader
  *   of the old state (sconv_kv_stage_conv).  W == 1 has no state: no-op.
@@ -362,7 +367,9 @@ SCONV_KV_API int sconv_kv_stage_rmsnorm(
 SCONV_KV_API int sconv_kv_stage_scatter(
     const void* z, int64_t num_tokens, int num_kv_heads, int head_dim,
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
-    const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream);
+    const sconv_kv_cache_layout_t* layout, const int32_t* cu_seqlens,
+    int num_seqs, int W, const int32_t* state_indices,
+    int64_t state_pool_size, int* err_flag, void* stream);
 
 SCONV_KV_API int sconv_kv_stage_state_update(
     const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
@@ -375,15 +382,21 @@ SCONV_KV_API int sconv_kv_stage_state_update(
  * (conv, rmsnorm, scatter, state update, in that order on `stream`), their
  * bf16 intermediates y and z placed in a scratch buffer that the library
  * holds in static device memory (SCONV_KV_NOALLOC_SCRATCH_BYTES per device,
- * reserved when the library's module loads; its address is looked up once
- * per device).  The library allocates nothing on any call.
+ * reserved when the library's module loads; every call looks up its
+ * address in the current context, a host-side lookup that allocates
+ * nothing).  The library allocates nothing on any call.
  *
  * Arguments and results as for sconv_kv_prefill_varlen (bf16 caches), and
- * the results equal those of the four sconv_kv_stage_* calls.  The call
- * needs 2 * round_up_256(num_tokens * 2 * num_kv_heads * head_dim * 2)
- * bytes of scratch; a larger call returns SCONV_KV_ERR_SCRATCH before
- * enqueueing anything.  Calls share the one scratch buffer: they must be
- * ordered (one stream, or streams ordered by events).
+ * the results equal those of the four sconv_kv_stage_* calls (scatter given
+ * cu_seqlens, so a skipped sequence leaves its cache slots untouched).
+ * Every argument of all four stages is checked before the first launch:
+ * an argument error returns with nothing enqueued.  Only a CUDA launch
+ * failure (SCONV_KV_ERR_CUDA) can come after earlier stages were enqueued.
+ * The call needs 2 * round_up_256(num_tokens * 2 * num_kv_heads * head_dim
+ * * 2) bytes of scratch; a larger call returns SCONV_KV_ERR_SCRATCH before
+ * enqueueing anything.  Calls share the one scratch buffer, which keeps
+ * whatever the last call left in it: calls that overlap on the GPU race,
+ * so they must be ordered (one stream, or streams ordered by events).
  *
  * The source pages have no counterpart to this entry point: it is a
  * convenience of this library.

@@ -94,7 +94,8 @@ def _load(path):
     lib.sconv_kv_stage_conv.restype = i32
     lib.sconv_kv_stage_rmsnorm.argtypes = [vp, i64, vp, vp, f32, i32, i32, vp, vp]
     lib.sconv_kv_stage_rmsnorm.restype = i32
-    lib.sconv_kv_stage_scatter.argtypes = [vp, i64, i32, i32, vp, vp, vp, lp, ip, vp]
+    lib.sconv_kv_stage_scatter.argtypes = [vp, i64, i32, i32, vp, vp, vp, lp, vp, i32, i32,
+                                           vp, i64, ip, vp]
     lib.sconv_kv_stage_scatter.restype = i32
     lib.sconv_kv_stage_state_update.argtypes = [
         vp, vp, i64, i64, vp, i32, i32, i32, i32, vp, vp, i64, ip, vp]
@@ -459,13 +460,20 @@ def stage_rmsnorm(y, gamma_k, gamma_v, eps, num_kv_heads, z, stream=None):
                                        _stream(stream)), "sconv_kv_stage_rmsnorm")
 
 
-def stage_scatter(z, slot_mapping, k_cache, v_cache, err_flag=None, stream=None):
-    """Pass 3: cache[slot_mapping[t]] = z[t] (K half / V half)."""
+def stage_scatter(z, slot_mapping, k_cache, v_cache, err_flag=None, stream=None,
+                  cu_seqlens=None, W=1, state_indices=None, state_pool_size=0):
+    """Pass 3: cache[slot_mapping[t]] = z[t] (K half / V half).  With
+    cu_seqlens, the tokens of sequences the other stages skip (malformed
+    cu_seqlens entry; for W > 1 a state index outside the pool) are not
+    written."""
     lay = layout_of(k_cache)
     H, D = k_cache.shape[2], k_cache.shape[3]
+    S = cu_seqlens.shape[0] - 1 if cu_seqlens is not None else 0
     _check(_lib.sconv_kv_stage_scatter(_ptr(z), z.shape[0], H, D, _ptr(slot_mapping),
                                        _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
-                                       _ptr(err_flag), _stream(stream)), "sconv_kv_stage_scatter")
+                                       _ptr(cu_seqlens), S, int(W), _ptr(state_indices),
+                                       int(state_pool_size), _ptr(err_flag), _stream(stream)),
+           "sconv_kv_stage_scatter")
 
 
 def stage_state_update(k, v, cu_seqlens, W, conv_state, state_indices=None, err_flag=None,
@@ -503,6 +511,7 @@ def prepare_unfused(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
                                                 ctypes.c_float(eps), H, D, _ptr(z), sp)),
         PreparedCall("sconv_kv_stage_scatter", (_ptr(z), T, H, D, _ptr(slot_mapping),
                                                 _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay),
+                                                _ptr(cu_seqlens), S, W, _ptr(state_indices), pool,
                                                 _ptr(err_flag), sp), keep_alive=(lay,)),
         PreparedCall("sconv_kv_stage_state_update", (kp, vp, rs, T, _ptr(cu_seqlens), S, W, H, D,
                                                      st, _ptr(state_indices), pool,

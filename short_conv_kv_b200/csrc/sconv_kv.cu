@@ -109,6 +109,71 @@ int sm_count() {
   return n;
 }
 
+// Shared memory of one SM and the part of it each resident CTA reserves
+// (cached per device).
+void smem_per_sm(size_t* total, size_t* reserved_per_cta) {
+  static size_t cached_total[64] = {0}, cached_res[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    *total = 228 * 1024;
+    *reserved_per_cta = 1024;
+    return;
+  }
+  std::lock_guard<std::mutex> lock(g_cache_mutex);
+  if (!cached_total[dev]) {
+    int t = 0, r = 0;
+    if (cudaDeviceGetAttribute(&t, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        t <= 0)
+      t = 228 * 1024;
+    if (cudaDeviceGetAttribute(&r, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        r < 0)
+      r = 1024;
+    cudaGetLastError();
+    cached_total[dev] = static_cast<size_t>(t);
+    cached_res[dev] = static_cast<size_t>(r);
+  }
+  *total = cached_total[dev];
+  *reserved_per_cta = cached_res[dev];
+}
+
+// CTAs of `fn` that fit on one SM with `threads` threads and `smem` bytes of
+// dynamic shared memory (after the kernel has been opted into that size);
+// `fallback` if the query fails.  Cached per device, kernel and size.
+int resident_per_sm(const void* fn, int threads, size_t smem, int fallback) {
+  static const void* c_fn[256];
+  static int c_dev[256], c_threads[256], c_n[256];
+  static size_t c_smem[256];
+  static int n_cached = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fallback;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_cache_mutex);
+    for (int i = 0; i < n_cached; ++i)
+      if (c_fn[i] == fn && c_dev[i] == dev && c_threads[i] == threads && c_smem[i] == smem)
+        return c_n[i];
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    return fallback;
+  }
+  std::lock_guard<std::mutex> lock(g_cache_mutex);
+  if (n_cached < 256) {
+    c_fn[n_cached] = fn;
+    c_dev[n_cached] = dev;
+    c_threads[n_cached] = threads;
+    c_smem[n_cached] = smem;
+    c_n[n_cached] = n;
+    ++n_cached;
+  }
+  return n;
+}
+
 // Opt a kernel into `bytes` of dynamic shared memory (once per kernel and
 // size; host-side attribute, not a stream operation).
 bool smem_attr_set(const void* fn, size_t bytes) {
@@ -296,12 +361,30 @@ int prefill_impl(
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
   // + per-warp slot-offset tables + per-thread gammas
   G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes + sconv::kTmaGammaBytes;
-  G.cu_smem = num_seqs < sconv::kTmaCuSmemMax ? 1 : 0;
+  // cu_seqlens is staged in shared memory only while per_sm CTAs still fit
+  // on an SM with it (beyond that the CTAs read it from global memory):
+  // staging must never cost a resident CTA
+  const size_t smem_base = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 48;
+  const size_t cu_bytes = 4 * (static_cast<size_t>(num_seqs) + 1);
+  size_t sm_total = 0, sm_reserved = 0;
+  smem_per_sm(&sm_total, &sm_reserved);
+  G.cu_smem = (num_seqs < sconv::kTmaCuSmemMax &&
+               per_sm * (smem_base + cu_bytes + sm_reserved) <= sm_total) ? 1 : 0;
   G.timeout_ns = (opts && opts->wait_timeout_ns > 0)
                      ? static_cast<unsigned long long>(opts->wait_timeout_ns)
                      : 1000000000ull;
   G.withhold_first = (opts && opts->withhold_first_copy) ? 1 : 0;
-  const int64_t resident = static_cast<int64_t>(sm_count()) * per_sm;
+  const size_t smem = smem_base + (G.cu_smem ? cu_bytes : 0);
+  if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
+    return SCONV_KV_ERR_CUDA;
+  }
+  const dim3 block(((G.slice + 31) / 32) * 32);
+  // persistent CTAs: as many as are resident at this shared-memory size
+  // (never more, or the rest would run as a second wave)
+  const int occ = resident_per_sm(reinterpret_cast<const void*>(fn), static_cast<int>(block.x),
+                                  smem, per_sm);
+  const int64_t resident = static_cast<int64_t>(sm_count()) * (occ < per_sm ? occ : per_sm);
   int64_t ctas = resident / ctas_y;
   const int64_t by_tokens = (num_tokens + sconv::kTmaRows - 1) / sconv::kTmaRows;
   if (ctas > by_tokens) ctas = by_tokens;
@@ -313,13 +396,6 @@ int prefill_impl(
   G.seq_cost = SCONV_PREFILL_SEQ_COST;
   G.cut_q = static_cast<int>(num_tokens / ctas);
   G.cut_r = static_cast<int>(num_tokens % ctas);
-  const size_t smem = static_cast<size_t>(G.smem_ring) + 16 * G.stages + 48 +
-                      (G.cu_smem ? 4 * static_cast<size_t>(num_seqs + 1) : 0);
-  if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
-    snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
-    return SCONV_KV_ERR_CUDA;
-  }
-  const dim3 block(((G.slice + 31) / 32) * 32);
   void* args[] = {&P, &G};
   return launch(reinterpret_cast<const void*>(fn), dim3(G.ctas, ctas_y), block, args, smem,
                 stream);
@@ -456,22 +532,140 @@ int stage_launch(StageFn fn, int64_t work, sconv::StageParams* P, void* stream) 
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[SCONV_KV_NOALLOC_SCRATCH_BYTES];
 
-// Device address of the scratch on the current device, looked up once per
-// device (nullptr if the lookup fails).
+// Device address of the scratch in the current device's context, looked up
+// on every call (a host-side table lookup, no allocation): a cached address
+// could outlive its context (cudaDeviceReset, or a caller that switches
+// driver contexts).  nullptr if the lookup fails.
 unsigned char* noalloc_scratch() {
-  static unsigned char* cached[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(g_cache_mutex);
-  if (!cached[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    cached[dev] = static_cast<unsigned char*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return cached[dev];
+  return static_cast<unsigned char*>(p);
+}
+
+// ---- unfused stages: argument checks (nothing enqueued) and launches
+
+int prep_stage_conv(const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+                    const int32_t* cu_seqlens, int num_seqs, const void* conv_w_k,
+                    const void* conv_w_v, int W, int num_kv_heads, int head_dim,
+                    const void* conv_state, const int32_t* state_indices,
+                    int64_t state_pool_size, void* y, int* err_flag, sconv::StageParams* P) {
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, P);
+  if (st) return st;
+  if (!k || !v || !cu_seqlens || !conv_w_k || !conv_w_v || !y || (W > 1 && !conv_state))
+    return SCONV_KV_ERR_NULL;
+  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P->C)
+    return SCONV_KV_ERR_SHAPE;
+  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_w_k) ||
+      !aligned16(conv_w_v) || !aligned16(y) || (conv_state && !aligned16(conv_state)))
+    return SCONV_KV_ERR_ALIGN;
+  P->k = static_cast<const uint16_t*>(k);
+  P->v = static_cast<const uint16_t*>(v);
+  P->row_stride = row_stride;
+  P->cu_seqlens = cu_seqlens;
+  P->num_seqs = num_seqs;
+  P->w_k = static_cast<const uint16_t*>(conv_w_k);
+  P->w_v = static_cast<const uint16_t*>(conv_w_v);
+  P->W = W;
+  P->state = const_cast<uint16_t*>(static_cast<const uint16_t*>(conv_state));
+  P->state_indices = state_indices;
+  P->pool = state_pool_size;
+  P->y = static_cast<uint16_t*>(y);
+  P->err = err_flag;
+  return SCONV_KV_OK;
+}
+
+int prep_stage_rmsnorm(const void* y, int64_t num_tokens, const float* gamma_k,
+                       const float* gamma_v, float eps, int num_kv_heads, int head_dim, void* z,
+                       sconv::StageParams* P) {
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, P);
+  if (st) return st;
+  if (!y || !gamma_k || !gamma_v || !z) return SCONV_KV_ERR_NULL;
+  if (!aligned16(y) || !aligned16(z) || !aligned16(gamma_k) || !aligned16(gamma_v))
+    return SCONV_KV_ERR_ALIGN;
+  P->y = const_cast<uint16_t*>(static_cast<const uint16_t*>(y));
+  P->z = static_cast<uint16_t*>(z);
+  P->gamma_k = gamma_k;
+  P->gamma_v = gamma_v;
+  P->eps = eps;
+  return SCONV_KV_OK;
+}
+
+int prep_stage_scatter(const void* z, int64_t num_tokens, int num_kv_heads, int head_dim,
+                       const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                       const sconv_kv_cache_layout_t* layout, const int32_t* cu_seqlens,
+                       int num_seqs, int W, const int32_t* state_indices,
+                       int64_t state_pool_size, int* err_flag, sconv::StageParams* P) {
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, P);
+  if (st) return st;
+  if (!z || !slot_mapping || !k_cache || !v_cache || !layout) return SCONV_KV_ERR_NULL;
+  if (cu_seqlens && (num_seqs < 1 || W < 1 || W > SCONV_KV_MAX_W || state_pool_size < 0))
+    return SCONV_KV_ERR_SHAPE;
+  if (layout->num_kv_heads != num_kv_heads || layout->head_dim != head_dim ||
+      layout->num_pages < 0 || layout->page_size < 1 || layout->stride_head < head_dim ||
+      layout->stride_slot < 1 || layout->stride_page < 1)
+    return SCONV_KV_ERR_SHAPE;
+  if (!aligned16(z) || !aligned16(k_cache) || !aligned16(v_cache) || layout->stride_head % 8 ||
+      layout->stride_slot % 8 || layout->stride_page % 8)
+    return SCONV_KV_ERR_ALIGN;
+  P->z = const_cast<uint16_t*>(static_cast<const uint16_t*>(z));
+  P->slots = slot_mapping;
+  P->k_cache = static_cast<uint16_t*>(k_cache);
+  P->v_cache = static_cast<uint16_t*>(v_cache);
+  P->num_slots = layout->num_pages * layout->page_size;
+  P->page_size = layout->page_size;
+  P->stride_page = layout->stride_page;
+  P->stride_slot = layout->stride_slot;
+  P->stride_head = layout->stride_head;
+  P->cu_seqlens = cu_seqlens;
+  P->num_seqs = cu_seqlens ? num_seqs : 0;
+  P->W = cu_seqlens ? W : 1;
+  P->state_indices = state_indices;
+  P->pool = state_pool_size;
+  P->err = err_flag;
+  return SCONV_KV_OK;
+}
+
+int prep_stage_state(const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
+                     const int32_t* cu_seqlens, int num_seqs, int W, int num_kv_heads,
+                     int head_dim, void* conv_state, const int32_t* state_indices,
+                     int64_t state_pool_size, int* err_flag, sconv::StageParams* P) {
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, P);
+  if (st) return st;
+  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P->C)
+    return SCONV_KV_ERR_SHAPE;
+  if (W == 1 || num_seqs == 0) return SCONV_KV_OK;  // no state rows: nothing to launch
+  if (!k || !v || !cu_seqlens || !conv_state) return SCONV_KV_ERR_NULL;
+  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_state))
+    return SCONV_KV_ERR_ALIGN;
+  P->k = static_cast<const uint16_t*>(k);
+  P->v = static_cast<const uint16_t*>(v);
+  P->row_stride = row_stride;
+  P->cu_seqlens = cu_seqlens;
+  P->num_seqs = num_seqs;
+  P->W = W;
+  P->state = static_cast<uint16_t*>(conv_state);
+  P->state_indices = state_indices;
+  P->pool = state_pool_size;
+  P->err = err_flag;
+  return SCONV_KV_OK;
+}
+
+int launch_stage_conv(sconv::StageParams* P, void* stream) {
+  return stage_launch(stage_conv_by_w(P->W), P->num_tokens * P->NG, P, stream);
+}
+int launch_stage_rmsnorm(sconv::StageParams* P, void* stream) {
+  return stage_launch(stage_rmsnorm_by_d(P->D), P->num_tokens * P->NG, P, stream);
+}
+int launch_stage_scatter(sconv::StageParams* P, void* stream) {
+  return stage_launch(sconv::stage_scatter_kernel, P->num_tokens * P->NG, P, stream);
+}
+int launch_stage_state(sconv::StageParams* P, void* stream) {
+  if (P->W <= 1 || P->num_seqs == 0) return SCONV_KV_OK;
+  return stage_launch(stage_state_by_w(P->W), static_cast<int64_t>(P->num_seqs) * P->NG, P,
+                      stream);
 }
 
 }  // namespace
@@ -631,8 +825,13 @@ int sconv_kv_unfused_step_noalloc(
     const int32_t* state_indices, int64_t state_pool_size,
     const int64_t* slot_mapping, void* k_cache, void* v_cache,
     const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
-  if (num_tokens < 0 || num_kv_heads < 1 || head_dim < 1) return SCONV_KV_ERR_SHAPE;
+  // shape limits first, so the scratch size below cannot overflow
+  sconv::StageParams shape;
+  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &shape);
+  if (st) return st;
+  if (num_seqs < 0) return SCONV_KV_ERR_SHAPE;
   if (num_tokens == 0 || num_seqs == 0) return SCONV_KV_OK;
+  // num_tokens < 2^31, channels <= 2^24: the product stays below 2^58
   const int64_t bytes = num_tokens * 2 * static_cast<int64_t>(num_kv_heads) * head_dim * 2;
   const int64_t part = (bytes + 255) / 256 * 256;
   if (2 * part > SCONV_KV_NOALLOC_SCRATCH_BYTES) return SCONV_KV_ERR_SCRATCH;
@@ -643,19 +842,26 @@ int sconv_kv_unfused_step_noalloc(
   }
   void* y = scratch;
   void* z = scratch + part;
-  int st = sconv_kv_stage_conv(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k,
-                               conv_w_v, W, num_kv_heads, head_dim, conv_state, state_indices,
-                               state_pool_size, y, err_flag, stream);
+  // every stage's arguments are checked before the first launch, so an
+  // argument error leaves nothing enqueued
+  sconv::StageParams Pc, Pn, Ps, Pu;
+  st = prep_stage_conv(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                       W, num_kv_heads, head_dim, conv_state, state_indices, state_pool_size, y,
+                       err_flag, &Pc);
   if (st) return st;
-  st = sconv_kv_stage_rmsnorm(y, num_tokens, gamma_k, gamma_v, eps, num_kv_heads, head_dim, z,
-                              stream);
+  st = prep_stage_rmsnorm(y, num_tokens, gamma_k, gamma_v, eps, num_kv_heads, head_dim, z, &Pn);
   if (st) return st;
-  st = sconv_kv_stage_scatter(z, num_tokens, num_kv_heads, head_dim, slot_mapping, k_cache,
-                              v_cache, layout, err_flag, stream);
+  st = prep_stage_scatter(z, num_tokens, num_kv_heads, head_dim, slot_mapping, k_cache, v_cache,
+                          layout, cu_seqlens, num_seqs, W, state_indices, state_pool_size,
+                          err_flag, &Ps);
   if (st) return st;
-  return sconv_kv_stage_state_update(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, W,
-                                     num_kv_heads, head_dim, conv_state, state_indices,
-                                     state_pool_size, err_flag, stream);
+  st = prep_stage_state(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, W, num_kv_heads,
+                        head_dim, conv_state, state_indices, state_pool_size, err_flag, &Pu);
+  if (st) return st;
+  if ((st = launch_stage_conv(&Pc, stream))) return st;
+  if ((st = launch_stage_rmsnorm(&Pn, stream))) return st;
+  if ((st = launch_stage_scatter(&Ps, stream))) return st;
+  return launch_stage_state(&Pu, stream);
 }
 
 int sconv_kv_stage_conv(const void* k, const void* v, int64_t row_stride, int64_t num_tokens,
@@ -667,27 +873,11 @@ int sconv_kv_stage_conv(const void* k, const void* v, int64_t row_stride, int64_
   int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
   if (st) return st;
   if (num_tokens == 0 || num_seqs == 0) return SCONV_KV_OK;
-  if (!k || !v || !cu_seqlens || !conv_w_k || !conv_w_v || !y || (W > 1 && !conv_state))
-    return SCONV_KV_ERR_NULL;
-  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P.C)
-    return SCONV_KV_ERR_SHAPE;
-  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_w_k) ||
-      !aligned16(conv_w_v) || !aligned16(y) || (conv_state && !aligned16(conv_state)))
-    return SCONV_KV_ERR_ALIGN;
-  P.k = static_cast<const uint16_t*>(k);
-  P.v = static_cast<const uint16_t*>(v);
-  P.row_stride = row_stride;
-  P.cu_seqlens = cu_seqlens;
-  P.num_seqs = num_seqs;
-  P.w_k = static_cast<const uint16_t*>(conv_w_k);
-  P.w_v = static_cast<const uint16_t*>(conv_w_v);
-  P.W = W;
-  P.state = const_cast<uint16_t*>(static_cast<const uint16_t*>(conv_state));
-  P.state_indices = state_indices;
-  P.pool = state_pool_size;
-  P.y = static_cast<uint16_t*>(y);
-  P.err = err_flag;
-  return stage_launch(stage_conv_by_w(W), num_tokens * P.NG, &P, stream);
+  st = prep_stage_conv(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, conv_w_k, conv_w_v,
+                       W, num_kv_heads, head_dim, conv_state, state_indices, state_pool_size, y,
+                       err_flag, &P);
+  if (st) return st;
+  return launch_stage_conv(&P, stream);
 }
 
 int sconv_kv_stage_rmsnorm(const void* y, int64_t num_tokens, const float* gamma_k,
@@ -697,43 +887,25 @@ int sconv_kv_stage_rmsnorm(const void* y, int64_t num_tokens, const float* gamma
   int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
   if (st) return st;
   if (num_tokens == 0) return SCONV_KV_OK;
-  if (!y || !gamma_k || !gamma_v || !z) return SCONV_KV_ERR_NULL;
-  if (!aligned16(y) || !aligned16(z) || !aligned16(gamma_k) || !aligned16(gamma_v))
-    return SCONV_KV_ERR_ALIGN;
-  P.y = const_cast<uint16_t*>(static_cast<const uint16_t*>(y));
-  P.z = static_cast<uint16_t*>(z);
-  P.gamma_k = gamma_k;
-  P.gamma_v = gamma_v;
-  P.eps = eps;
-  return stage_launch(stage_rmsnorm_by_d(head_dim), num_tokens * P.NG, &P, stream);
+  st = prep_stage_rmsnorm(y, num_tokens, gamma_k, gamma_v, eps, num_kv_heads, head_dim, z, &P);
+  if (st) return st;
+  return launch_stage_rmsnorm(&P, stream);
 }
 
 int sconv_kv_stage_scatter(const void* z, int64_t num_tokens, int num_kv_heads, int head_dim,
                            const int64_t* slot_mapping, void* k_cache, void* v_cache,
-                           const sconv_kv_cache_layout_t* layout, int* err_flag, void* stream) {
+                           const sconv_kv_cache_layout_t* layout, const int32_t* cu_seqlens,
+                           int num_seqs, int W, const int32_t* state_indices,
+                           int64_t state_pool_size, int* err_flag, void* stream) {
   sconv::StageParams P;
   int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
   if (st) return st;
   if (num_tokens == 0) return SCONV_KV_OK;
-  if (!z || !slot_mapping || !k_cache || !v_cache || !layout) return SCONV_KV_ERR_NULL;
-  if (layout->num_kv_heads != num_kv_heads || layout->head_dim != head_dim ||
-      layout->num_pages < 0 || layout->page_size < 1 || layout->stride_head < head_dim ||
-      layout->stride_slot < 1 || layout->stride_page < 1)
-    return SCONV_KV_ERR_SHAPE;
-  if (!aligned16(z) || !aligned16(k_cache) || !aligned16(v_cache) || layout->stride_head % 8 ||
-      layout->stride_slot % 8 || layout->stride_page % 8)
-    return SCONV_KV_ERR_ALIGN;
-  P.z = const_cast<uint16_t*>(static_cast<const uint16_t*>(z));
-  P.slots = slot_mapping;
-  P.k_cache = static_cast<uint16_t*>(k_cache);
-  P.v_cache = static_cast<uint16_t*>(v_cache);
-  P.num_slots = layout->num_pages * layout->page_size;
-  P.page_size = layout->page_size;
-  P.stride_page = layout->stride_page;
-  P.stride_slot = layout->stride_slot;
-  P.stride_head = layout->stride_head;
-  P.err = err_flag;
-  return stage_launch(sconv::stage_scatter_kernel, num_tokens * P.NG, &P, stream);
+  st = prep_stage_scatter(z, num_tokens, num_kv_heads, head_dim, slot_mapping, k_cache, v_cache,
+                          layout, cu_seqlens, num_seqs, W, state_indices, state_pool_size,
+                          err_flag, &P);
+  if (st) return st;
+  return launch_stage_scatter(&P, stream);
 }
 
 int sconv_kv_stage_state_update(const void* k, const void* v, int64_t row_stride,
@@ -742,25 +914,10 @@ int sconv_kv_stage_state_update(const void* k, const void* v, int64_t row_stride
                                 const int32_t* state_indices, int64_t state_pool_size,
                                 int* err_flag, void* stream) {
   sconv::StageParams P;
-  int st = stage_shape(num_kv_heads, head_dim, num_tokens, &P);
+  int st = prep_stage_state(k, v, row_stride, num_tokens, cu_seqlens, num_seqs, W, num_kv_heads,
+                            head_dim, conv_state, state_indices, state_pool_size, err_flag, &P);
   if (st) return st;
-  if (W < 1 || W > SCONV_KV_MAX_W || num_seqs < 0 || state_pool_size < 0 || row_stride < P.C)
-    return SCONV_KV_ERR_SHAPE;
-  if (W == 1 || num_seqs == 0) return SCONV_KV_OK;  // no state rows
-  if (!k || !v || !cu_seqlens || !conv_state) return SCONV_KV_ERR_NULL;
-  if (row_stride % 8 || !aligned16(k) || !aligned16(v) || !aligned16(conv_state))
-    return SCONV_KV_ERR_ALIGN;
-  P.k = static_cast<const uint16_t*>(k);
-  P.v = static_cast<const uint16_t*>(v);
-  P.row_stride = row_stride;
-  P.cu_seqlens = cu_seqlens;
-  P.num_seqs = num_seqs;
-  P.W = W;
-  P.state = static_cast<uint16_t*>(conv_state);
-  P.state_indices = state_indices;
-  P.pool = state_pool_size;
-  P.err = err_flag;
-  return stage_launch(stage_state_by_w(W), static_cast<int64_t>(num_seqs) * P.NG, &P, stream);
+  return launch_stage_state(&P, stream);
 }
 
 }  // extern "C"

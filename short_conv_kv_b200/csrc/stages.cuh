@@ -168,7 +168,12 @@ __global__ void __launch_bounds__(256) stage_rmsnorm_kernel(const StageParams P)
 }
 
 // Pass 3: cache[slot_mapping[t]] = z[t] (K half into k_cache, V half into
-// v_cache); slot < 0 skips the token, slot >= num_slots is flagged.
+// v_cache); slot < 0 skips the token, slot >= num_slots is flagged.  When
+// cu_seqlens is given, the tokens of a sequence that the fused step would
+// skip (malformed cu_seqlens entry; for W > 1 a state index outside the
+// pool) are not written either, so the chain leaves the same cache slots
+// untouched as the fused kernels (the conv and state passes raise the
+// flags).
 __global__ void __launch_bounds__(256) stage_scatter_kernel(const StageParams P) {
   grid_dependency_wait();
   const int64_t total = P.num_tokens * P.NG;
@@ -179,6 +184,16 @@ __global__ void __launch_bounds__(256) stage_scatter_kernel(const StageParams P)
     const int g = static_cast<int>(idx - t * P.NG);
     const int64_t slot = __ldg(P.slots + t);
     if (slot < 0) continue;
+    if (P.cu_seqlens) {
+      const int i = stage_seq_of(P.cu_seqlens, P.num_seqs, t);
+      const int64_t a = __ldg(P.cu_seqlens + i), e = __ldg(P.cu_seqlens + i + 1);
+      if (!(a >= 0 && a <= t && t < e && e <= P.num_tokens)) continue;
+      if (P.W > 1) {
+        const int64_t si =
+            P.state_indices ? static_cast<int64_t>(__ldg(P.state_indices + i)) : i;
+        if (si < 0 || si >= P.pool) continue;
+      }
+    }
     if (slot >= P.num_slots) {
       if (g == 0) raise_flag(P.err, kFlagSlotRange);
       continue;

@@ -173,3 +173,27 @@ def test_unfused_chain_matches_oracle(lengths, W):
         err = np.abs(got - zz)
         assert (err <= np.maximum(gu.ABS_TOL, gu.REL_TOL * np.abs(zz))).all(), (which, err.max())
     assert np.array_equal(wl.bits(st.cpu()), ref["conv_state"])
+
+
+def test_stage_scatter_skips_flagged_sequences():
+    """Given cu_seqlens, scatter leaves the slots of a sequence with a bad
+    state index (W > 1) untouched, as the fused step does; without it,
+    every token is written."""
+    bd = _bd()
+    b = wl.make_prefill([20, 33, 11], Hkv=2, D=64, W=4, seed=2660, state="zero", page_size=16,
+                        spare_pages=2, pool_size=3, state_indices=[0, 7, 2])
+    g = torch.Generator().manual_seed(2661)
+    z = gu.dev(torch.randn(b.num_tokens, 2 * b.C, generator=g).to(torch.bfloat16))
+    sent = np.uint16(wl.SENTINEL_BITS)
+    sm = b.slot_mapping.numpy()
+    for with_seqs in (True, False):
+        kc, vc = gu.dev(b.empty_cache()), gu.dev(b.empty_cache())
+        kw = dict(cu_seqlens=gu.dev(b.cu_seqlens), W=b.W, state_indices=gu.dev(b.state_indices),
+                  state_pool_size=3) if with_seqs else {}
+        bd.stage_scatter(z, gu.dev(b.slot_mapping), kc, vc, **kw)
+        torch.cuda.synchronize()
+        for cache in (kc, vc):
+            rows = wl.bits(cache.cpu()).reshape(-1, b.C)
+            untouched = np.all(rows == sent, axis=1)
+            assert untouched[sm[20:53]].all() == with_seqs
+            assert not untouched[sm[:20]].any() and not untouched[sm[53:]].any()
