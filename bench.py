@@ -193,6 +193,12 @@ class Workload:
         self.ring = name.endswith("_ring")  # ring-buffer conv_state (decode)
         self.name, self.rank = name, rank
         self.launches_per_step = 1
+        # prefill calls with the state-only dependency (the previous launch
+        # writes none of a call's inputs but conv_state): set by the caller
+        self.chain_overlap = False
+        # decode calls with the independent-state promise (the previous
+        # launch writes none of a call's state rows): set by the caller
+        self.early_state = False
         seed_shift = 97 * rank
         if name == "single":
             self.kind, self.batches = "prefill", [wl.single(seed=2000 + seed_shift)]
@@ -319,21 +325,23 @@ class Workload:
             return self.binding.prepare_decode_mxfp8(
                 a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
                 a["eps"], a["conv_state"], a["slot_mapping"], a["k_data"], a["k_scale"],
-                a["v_data"], a["v_scale"], stream=stream)
+                a["v_data"], a["v_scale"], stream=stream, independent_state=self.early_state)
         if self.mx:
             return self.binding.prepare_prefill_varlen_mxfp8(
                 a["k"], a["v"], a["cu_seqlens"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"],
                 a["gamma_v"], a["eps"], a["conv_state"], a["slot_mapping"], a["k_data"],
-                a["k_scale"], a["v_data"], a["v_scale"], stream=stream)
+                a["k_scale"], a["v_data"], a["v_scale"], stream=stream,
+                state_only_dependency=self.chain_overlap)
         if self.kind == "decode":
             return self.binding.prepare_decode(
                 a["k"], a["v"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"], a["gamma_v"],
                 a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"], a["v_cache"],
-                stream=stream, state_positions=a.get("state_positions"))
+                stream=stream, state_positions=a.get("state_positions"),
+                independent_state=self.early_state)
         return self.binding.prepare_prefill_varlen(
             a["k"], a["v"], a["cu_seqlens"], a["conv_w_k"], a["conv_w_v"], a["gamma_k"],
             a["gamma_v"], a["eps"], a["conv_state"], a["slot_mapping"], a["k_cache"],
-            a["v_cache"], stream=stream)
+            a["v_cache"], stream=stream, state_only_dependency=self.chain_overlap)
 
     def kernel_tag(self):
         tag = {"prefill": "prefill_tma_kernel", "long": "prefill_tma_kernel",
@@ -627,6 +635,24 @@ SIDE_MIN_MS = 20.0     # timed region per side workload, at least
 SIDE_MAX_LAUNCHES = 2500
 
 
+def time_isolated_launch(work, dev, reps=7):
+    """Median time of one launch on an idle GPU (synchronised before and
+    after, CUDA events around the single launch): the time a call takes
+    when nothing overlaps it, set against the chain's time per launch."""
+    stream = torch.cuda.Stream(device=dev)
+    times = []
+    for i in range(reps):
+        call = work.prepared(i, stream)
+        s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s_ev.record(stream)
+        call()
+        e_ev.record(stream)
+        e_ev.synchronize()
+        times.append(s_ev.elapsed_time(e_ev))
+    return statistics.median(times)
+
+
 def line_roofline(work, kern_ms, peaks, peak_src, traffic):
     achieved = work.bytes_per_launch / (kern_ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -674,6 +700,11 @@ def run_ours(args):
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
     work = Workload(args.workload, rank)
+    # consecutive chunks of one sequence are the case the state-only
+    # dependency is for: the long-context workload promises it by default
+    work.chain_overlap = work.kind != "decode" and (
+        args.chain_overlap or (work.kind == "long" and not args.no_chain_overlap))
+    work.early_state = args.early_state and work.kind == "decode"
     work.setup(dev)
     K, Wu = args.steps, args.warmup
     lps = work.launches_per_step
@@ -690,6 +721,23 @@ def run_ours(args):
         return
     ms_per_step = total_ms / K
     kern_ms = total_ms / (K * lps)  # average launch duration
+    chain = None
+    if lps > 1:
+        iso_ms = max_over_ranks(time_isolated_launch(work, dev), world)
+        chain = {"launches_per_step": lps, "ms_per_step": ms_per_step,
+                 "isolated_launch_ms": iso_ms,
+                 "step_vs_launches_alone": ms_per_step / (lps * iso_ms),
+                 "state_only_dependency": work.chain_overlap,
+                 "note": "the step's launches back to back (state carried) against as many "
+                         "launches each timed alone on an idle GPU"}
+        if work.chain_overlap:
+            # the same chain with every CTA waiting for the previous launch
+            work.chain_overlap = False
+            t2, _ = time_graph(work, K, Wu, dev, world, local)
+            work.chain_overlap = True
+            t2 = max_over_ranks(t2, world)
+            chain["without_state_only_dependency"] = {
+                "ms_per_step": t2 / K, "ms_per_launch": t2 / (K * lps)}
     value = world * work.tokens_per_step * K / (total_ms / 1e3)
     launches = K * lps
     e2e = None
@@ -746,10 +794,14 @@ def run_ours(args):
                        "parallelism": f"{world} independent replicas (sequence sharding, no collective)",
                        "l2": f"inputs rotate over {work.rotation} buffer sets "
                              f"({work.rotation * work.bytes_per_launch / 1e6:.0f} MB) > L2",
-                       "timing": "K steps in one CUDA graph replay, CUDA events around the replay"},
+                       "timing": "K steps in one CUDA graph replay, CUDA events around the replay",
+                       "calls": ("prefill calls promise the state-only dependency (the previous "
+                                 "launch writes none of a call's inputs but conv_state)"
+                                 if work.chain_overlap else "default calls")},
             "roofline": line_roofline(work, kern_ms, peaks, peak_src,
                                       profile_traffic(f"{work.kernel_tag()}_{args.workload}")),
             "configs": configs,
+            "chain": chain,
             "cpu_baseline": cpu,
             "unfused_chain": unfused,
             "e2e": e2e,
@@ -851,6 +903,16 @@ def main():
                     help="skip timing the unfused four-kernel chain (context only)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip timing the side workloads of the `configs` key")
+    ap.add_argument("--chain-overlap", action="store_true",
+                    help="prefill calls promise the state-only dependency (consecutive "
+                         "launches overlap; see include/sconv_kv.h); on by default for the "
+                         "long-context workload")
+    ap.add_argument("--no-chain-overlap", action="store_true",
+                    help="the long-context workload's calls without that promise")
+    ap.add_argument("--early-state", action="store_true",
+                    help="decode calls promise an independent state (each launch's state "
+                         "rows are not written by the launch before it; see "
+                         "include/sconv_kv.h)")
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket the timed replay with cudaProfilerStart/Stop and run nothing "
                          "else (for a range capture of the DRAM counters)")

@@ -263,15 +263,53 @@ SCONV_KV_API int sconv_kv_decode_mxfp8(
  *                     wait_timeout_ns and the timeout path above runs: a
  *                     wait on something that nothing completes, with no
  *                     fault.  The output of such a call is incomplete.
+ *  state_only_dependency  prefill only (decode ignores it).  Nonzero is a
+ *                     promise by the caller: the kernel enqueued just
+ *                     before this call on `stream` writes none of this
+ *                     call's inputs except conv_state, and none of the
+ *                     cache slots this call writes -- as when consecutive
+ *                     chunks of one long sequence are prefilled back to
+ *                     back (1M-token context: aib.vote English news item,
+ *                     paragraph 1; Inkling-Small cookbook, section 3.6).
+ *                     The call's CTAs are launched early (programmatic
+ *                     dependent launch) as usual, but only a CTA that
+ *                     reads or writes a conv_state row waits for that
+ *                     previous kernel to complete before it does so; every
+ *                     other CTA streams its rows and writes its cache slots
+ *                     at once, overlapping the previous kernel's tail.
+ *                     Every CTA still waits for the previous kernel before
+ *                     it lets the next one launch and before it exits, so
+ *                     ordering along the stream is kept.  0 (default): every
+ *                     CTA waits before its first global access.  Inputs
+ *                     produced by the previous kernel (e.g. a projection
+ *                     launched right before this call) break the promise:
+ *                     leave it 0 then.
+ *  independent_state  decode only (prefill ignores it).  Nonzero is a
+ *                     promise by the caller: the kernel enqueued just
+ *                     before this call on `stream` writes none of this
+ *                     call's inputs except k and v -- as when that kernel is
+ *                     the K/V projection of this very decode step -- and
+ *                     neither reads nor writes the conv_state rows or cache
+ *                     slots this call writes.  Each CTA then reads its
+ *                     index tables and requests its first sequence's W-1
+ *                     state rows before it waits for that kernel
+ *                     (programmatic dependent launch); only the K/V rows
+ *                     wait.  Every CTA waits before anything is written,
+ *                     before the next kernel may launch and before it
+ *                     exits.  0 (default): every CTA waits before its first
+ *                     global access.
  *
- * The pages fix neither (their norm is only "normalization" and the state
- * pool's layout is not given); both are layouts a serving runtime may use.
+ * The pages fix neither of the two layouts (their norm is only
+ * "normalization" and the state pool's layout is not given); both are
+ * layouts a serving runtime may use.
  */
 typedef struct sconv_kv_options_t {
   int64_t gamma_head_stride;
   const int64_t* state_positions;
   int64_t wait_timeout_ns;
   int64_t withhold_first_copy;
+  int64_t state_only_dependency;
+  int64_t independent_state;
 } sconv_kv_options_t;
 
 SCONV_KV_API int sconv_kv_prefill_varlen_ex(

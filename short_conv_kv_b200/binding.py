@@ -33,7 +33,8 @@ class CacheLayout(ctypes.Structure):
 class Options(ctypes.Structure):
     """sconv_kv_options_t: per-head gamma stride and ring-state positions."""
     _fields_ = [("gamma_head_stride", ctypes.c_int64), ("state_positions", ctypes.c_void_p),
-                ("wait_timeout_ns", ctypes.c_int64), ("withhold_first_copy", ctypes.c_int64)]
+                ("wait_timeout_ns", ctypes.c_int64), ("withhold_first_copy", ctypes.c_int64),
+                ("state_only_dependency", ctypes.c_int64), ("independent_state", ctypes.c_int64)]
 
 
 class SconvKVError(RuntimeError):
@@ -161,14 +162,20 @@ def _stream(stream):
     return int(stream)
 
 
-def _options(gamma_k, state_positions, wait_timeout_ns=None, withhold_first_copy=False):
+def _options(gamma_k, state_positions, wait_timeout_ns=None, withhold_first_copy=False,
+             state_only_dependency=False, independent_state=False):
     """Options struct for the _ex entry points, or None for the defaults
-    (gamma [D] shared by every head, linear state, 1 s wait limit).  gamma
-    [Hkv, D] selects per-head gammas; state_positions (int64 [S] on the
-    device) a ring state; wait_timeout_ns the kernels' wait limit."""
+    (gamma [D] shared by every head, linear state, 1 s wait limit, every
+    CTA waiting for the previous kernel).  gamma [Hkv, D] selects per-head
+    gammas; state_positions (int64 [S] on the device) a ring state;
+    wait_timeout_ns the kernels' wait limit; state_only_dependency the
+    caller's promise that the previous kernel on the stream writes none of
+    this call's inputs but conv_state; independent_state (decode) the
+    promise that it writes none of them but k and v (see
+    include/sconv_kv.h)."""
     per_head = gamma_k is not None and gamma_k.dim() == 2
     if not per_head and state_positions is None and not wait_timeout_ns and \
-            not withhold_first_copy:
+            not withhold_first_copy and not state_only_dependency and not independent_state:
         return None
     if state_positions is not None and state_positions.dtype != torch.int64:
         raise TypeError("state_positions must be int64")
@@ -177,6 +184,8 @@ def _options(gamma_k, state_positions, wait_timeout_ns=None, withhold_first_copy
     o.state_positions = _ptr(state_positions)
     o.wait_timeout_ns = int(wait_timeout_ns or 0)
     o.withhold_first_copy = 1 if withhold_first_copy else 0
+    o.state_only_dependency = 1 if state_only_dependency else 0
+    o.independent_state = 1 if independent_state else 0
     return o
 
 
@@ -198,7 +207,7 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                    eps, conv_state, slot_mapping, k_cache, v_cache,
                    state_indices=None, err_flag=None, stream=None,
                    layout=None, state_positions=None, wait_timeout_ns=None,
-                   withhold_first_copy=False):
+                   withhold_first_copy=False, state_only_dependency=False):
     """Fused ShortConv K/V step over a packed varlen batch, on the GPU.
 
     k, v: bf16 [T, Hkv, D] (rows may be strided slices); cu_seqlens int32
@@ -223,7 +232,8 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
             float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
             _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_cache),
             _ptr(v_cache), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy)
+    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy,
+                    state_only_dependency)
     if opts is None:
         rc = _lib.sconv_kv_prefill_varlen(*args, _ptr(err_flag), _stream(stream))
     else:
@@ -236,7 +246,7 @@ def prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
 def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
            slot_mapping, k_cache, v_cache, state_indices=None, err_flag=None,
            stream=None, layout=None, state_positions=None, wait_timeout_ns=None,
-           withhold_first_copy=False):
+           withhold_first_copy=False, independent_state=False):
     """Fused ShortConv K/V decode step: one new token per sequence
     (k, v: bf16 [B, Hkv, D]); same other arguments as prefill_varlen."""
     kp, rs = _rows(k, "k")
@@ -252,7 +262,8 @@ def decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
             _ptr(gamma_v), float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
             _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy)
+    opts = _options(gamma_k, state_positions, wait_timeout_ns, withhold_first_copy,
+                    independent_state=independent_state)
     if opts is None:
         rc = _lib.sconv_kv_decode(*args, _ptr(err_flag), _stream(stream))
     else:
@@ -283,7 +294,8 @@ def _mx_layout(k_data, k_scale, v_data, v_scale):
 
 def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                          eps, conv_state, slot_mapping, k_data, k_scale, v_data, v_scale,
-                         state_indices=None, err_flag=None, stream=None, state_positions=None):
+                         state_indices=None, err_flag=None, stream=None, state_positions=None,
+                         state_only_dependency=False):
     """The fused step with the block-scaled MXFP8 cache store (E4M3 codes in
     k_data/v_data, one E8M0 scale byte per 32 channels in k_scale/v_scale)."""
     kp, rs = _rows(k, "k")
@@ -298,7 +310,7 @@ def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
             _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v), float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool, _ptr(slot_mapping),
             _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions)
+    opts = _options(gamma_k, state_positions, state_only_dependency=state_only_dependency)
     if opts is None:
         rc = _lib.sconv_kv_prefill_varlen_mxfp8(*args, _ptr(err_flag), _stream(stream))
     else:
@@ -310,7 +322,7 @@ def prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
 
 def decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
                  slot_mapping, k_data, k_scale, v_data, v_scale, state_indices=None,
-                 err_flag=None, stream=None, state_positions=None):
+                 err_flag=None, stream=None, state_positions=None, independent_state=False):
     """Decode step with the MXFP8 cache store (one new token per sequence)."""
     kp, rs = _rows(k, "k")
     vp, rs_v = _rows(v, "v")
@@ -324,7 +336,7 @@ def decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
             _ptr(gamma_v), float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
             _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
             _ptr(v_data), _ptr(v_scale), ctypes.byref(lay))
-    opts = _options(gamma_k, state_positions)
+    opts = _options(gamma_k, state_positions, independent_state=independent_state)
     if opts is None:
         rc = _lib.sconv_kv_decode_mxfp8(*args, _ptr(err_flag), _stream(stream))
     else:
@@ -354,32 +366,38 @@ class PreparedCall:
 def prepare_prefill_varlen(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k,
                            gamma_v, eps, conv_state, slot_mapping, k_cache,
                            v_cache, state_indices=None, err_flag=None,
-                           stream=None):
+                           stream=None, state_only_dependency=False):
     kp, rs = _rows(k, "k")
     vp, _ = _rows(v, "v")
     W = conv_w_k.shape[0]
     H, D = k_cache.shape[2], k_cache.shape[3]
     lay = layout_of(k_cache)
     pool = conv_state.shape[0] if conv_state is not None else 0
-    args = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+    head = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
             _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
             ctypes.c_float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
-            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
-            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
-    return PreparedCall("sconv_kv_prefill_varlen", args, keep_alive=(lay,))
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(lay))
+    opts = _options(gamma_k, None, state_only_dependency=state_only_dependency)
+    if opts is None:
+        return PreparedCall("sconv_kv_prefill_varlen", head + (_ptr(err_flag), _stream(stream)),
+                            keep_alive=(lay,))
+    return PreparedCall("sconv_kv_prefill_varlen_ex",
+                        head + (ctypes.byref(opts), _ptr(err_flag), _stream(stream)),
+                        keep_alive=(lay, opts))
 
 
 def prepare_decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
                    conv_state, slot_mapping, k_cache, v_cache,
-                   state_indices=None, err_flag=None, stream=None, state_positions=None):
+                   state_indices=None, err_flag=None, stream=None, state_positions=None,
+                   independent_state=False):
     kp, rs = _rows(k, "k")
     vp, _ = _rows(v, "v")
     W = conv_w_k.shape[0]
     H, D = k_cache.shape[2], k_cache.shape[3]
     lay = layout_of(k_cache)
     pool = conv_state.shape[0] if conv_state is not None else 0
-    opts = _options(gamma_k, state_positions)
+    opts = _options(gamma_k, state_positions, independent_state=independent_state)
     head = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v),
             _ptr(gamma_k), _ptr(gamma_v), ctypes.c_float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
@@ -394,36 +412,49 @@ def prepare_decode(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps,
 
 def prepare_prefill_varlen_mxfp8(k, v, cu_seqlens, conv_w_k, conv_w_v, gamma_k, gamma_v,
                                  eps, conv_state, slot_mapping, k_data, k_scale, v_data,
-                                 v_scale, state_indices=None, err_flag=None, stream=None):
+                                 v_scale, state_indices=None, err_flag=None, stream=None,
+                                 state_only_dependency=False):
     kp, rs = _rows(k, "k")
     vp, _ = _rows(v, "v")
     lay = _mx_layout(k_data, k_scale, v_data, v_scale)
     W = conv_w_k.shape[0]
     H, D = k_data.shape[2], k_data.shape[3]
     pool = conv_state.shape[0] if conv_state is not None else 0
-    args = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
+    head = (kp, vp, rs, k.shape[0], _ptr(cu_seqlens), cu_seqlens.shape[0] - 1,
             _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k), _ptr(gamma_v),
             ctypes.c_float(eps), W, H, D, _ptr(conv_state) if W > 1 else None,
             _ptr(state_indices), pool, _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale),
-            _ptr(v_data), _ptr(v_scale), ctypes.byref(lay), _ptr(err_flag), _stream(stream))
-    return PreparedCall("sconv_kv_prefill_varlen_mxfp8", args, keep_alive=(lay,))
+            _ptr(v_data), _ptr(v_scale), ctypes.byref(lay))
+    opts = _options(gamma_k, None, state_only_dependency=state_only_dependency)
+    if opts is None:
+        return PreparedCall("sconv_kv_prefill_varlen_mxfp8",
+                            head + (_ptr(err_flag), _stream(stream)), keep_alive=(lay,))
+    return PreparedCall("sconv_kv_prefill_varlen_mxfp8_ex",
+                        head + (ctypes.byref(opts), _ptr(err_flag), _stream(stream)),
+                        keep_alive=(lay, opts))
 
 
 def prepare_decode_mxfp8(k, v, conv_w_k, conv_w_v, gamma_k, gamma_v, eps, conv_state,
                          slot_mapping, k_data, k_scale, v_data, v_scale, state_indices=None,
-                         err_flag=None, stream=None):
+                         err_flag=None, stream=None, independent_state=False):
     kp, rs = _rows(k, "k")
     vp, _ = _rows(v, "v")
     lay = _mx_layout(k_data, k_scale, v_data, v_scale)
     W = conv_w_k.shape[0]
     H, D = k_data.shape[2], k_data.shape[3]
     pool = conv_state.shape[0] if conv_state is not None else 0
-    args = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
+    head = (kp, vp, rs, k.shape[0], _ptr(conv_w_k), _ptr(conv_w_v), _ptr(gamma_k),
             _ptr(gamma_v), ctypes.c_float(eps), W, H, D,
             _ptr(conv_state) if W > 1 else None, _ptr(state_indices), pool,
             _ptr(slot_mapping), _ptr(k_data), _ptr(k_scale), _ptr(v_data), _ptr(v_scale),
-            ctypes.byref(lay), _ptr(err_flag), _stream(stream))
-    return PreparedCall("sconv_kv_decode_mxfp8", args, keep_alive=(lay,))
+            ctypes.byref(lay))
+    opts = _options(gamma_k, None, independent_state=independent_state)
+    if opts is None:
+        return PreparedCall("sconv_kv_decode_mxfp8", head + (_ptr(err_flag), _stream(stream)),
+                            keep_alive=(lay,))
+    return PreparedCall("sconv_kv_decode_mxfp8_ex",
+                        head + (ctypes.byref(opts), _ptr(err_flag), _stream(stream)),
+                        keep_alive=(lay, opts))
 
 
 # ---------------------------------------------------------------- unfused stages

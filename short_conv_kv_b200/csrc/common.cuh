@@ -128,12 +128,25 @@ __device__ __forceinline__ int64_t slot_row_offset(const StepParams& P,
 
 // ---- MXFP8 (OCP Microscaling) block store: 32 channels = 4 lanes x 8.
 
-// Shared exponent of a block with largest magnitude `amax` (binary32):
-// floor(log2(amax)) - 8, the 8 being the exponent of E4M3's largest normal
-// (448 = 1.75 * 2^8); blocks whose amax is zero or subnormal take -127.
-__device__ __forceinline__ int mx_shared_exponent(float amax) {
-  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);  // biased
-  return e == 0 ? -127 : max(e - 127 - 8, -127);
+// E8M0 scale byte (s + 127) of a block whose largest magnitude is
+// `amax` (binary32, >= 0): the shared exponent s is floor(log2(amax)) - 8,
+// the 8 being the exponent of E4M3's largest normal (448 = 1.75 * 2^8),
+// and blocks whose amax is zero or subnormal take -127.  With e the biased
+// exponent of amax (its sign bit is clear), floor(log2(amax)) = e - 127
+// for a normal amax, so s + 127 = max(e - 8, 0) covers every case.
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+  return static_cast<uint32_t>(max(static_cast<int>(__float_as_uint(amax) >> 23) - 8, 0));
+}
+// 2^-s from the scale byte s + 127: biased exponent 254 - (s + 127).
+__device__ __forceinline__ float mx_inv_scale(uint32_t scale_byte) {
+  return __uint_as_float((254u - scale_byte) << 23);
+}
+// max(|a|, |b|, |c|) in one instruction (sm_100: three-input max with the
+// absolute-value modifier).
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Two binary32 -> two E4M3 codes (nearest even, saturating), low element
@@ -157,12 +170,13 @@ __device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool wr
   const float2 rr = make_float2(r, r);
   const float2 z[4] = {__fmul2_rn(t[0], rr), __fmul2_rn(t[1], rr), __fmul2_rn(t[2], rr),
                        __fmul2_rn(t[3], rr)};
-  float amax = fmaxf(fmaxf(fabsf(z[0].x), fabsf(z[0].y)), fmaxf(fabsf(z[1].x), fabsf(z[1].y)));
-  amax = fmaxf(amax, fmaxf(fmaxf(fabsf(z[2].x), fabsf(z[2].y)), fmaxf(fabsf(z[3].x), fabsf(z[3].y))));
+  const float m0 = max_abs3(z[0].x, z[0].y, z[1].x);
+  const float m1 = max_abs3(z[1].y, z[2].x, z[2].y);
+  float amax = fmaxf(m1, max_abs3(z[3].x, z[3].y, m0));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-  const int s = mx_shared_exponent(amax);
-  const float m = __uint_as_float(static_cast<uint32_t>(127 - s) << 23);  // 2^-s, exact
+  const uint32_t sb = mx_scale_byte(amax);
+  const float m = mx_inv_scale(sb);  // 2^-s, exact
   const float2 mm = make_float2(m, m);
   const float2 a = __fmul2_rn(z[0], mm), b = __fmul2_rn(z[1], mm);
   const float2 c = __fmul2_rn(z[2], mm), d = __fmul2_rn(z[3], mm);
@@ -175,8 +189,7 @@ __device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool wr
       "setp.ne.b32 r, %1, 0;\n\t"
       "@q st.global.cs.v2.u32 [%2], {%3, %4};\n\t"
       "@r st.global.cs.u8 [%5], %6;\n\t}" ::"r"(static_cast<int>(write)),
-      "r"(static_cast<int>(scale_writer)), "l"(data), "r"(w0), "r"(w1), "l"(scale),
-      "r"(static_cast<uint32_t>(s + 127))
+      "r"(static_cast<int>(scale_writer)), "l"(data), "r"(w0), "r"(w1), "l"(scale), "r"(sb)
       : "memory");
 }
 

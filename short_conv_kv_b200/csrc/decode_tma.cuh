@@ -29,6 +29,9 @@
 namespace sconv {
 
 constexpr int kDecMaxSeqs = 64;  // sequences per CTA (prologue index tables)
+#ifndef SCONV_DECODE_EARLY_STAGES
+#define SCONV_DECODE_EARLY_STAGES 1  // early state fetch: sequences requested before the wait
+#endif
 
 struct DecGeom {
   int slice;      // channel groups per full slice (min(NG, 256))
@@ -36,6 +39,7 @@ struct DecGeom {
   int ctas;       // CTAs along the batch
   int withhold_first;  // testing: the first sequence's copies are never made
   int smem_ring;  // bytes of the ring
+  int state_early;  // first sequence's state rows requested before the dependency wait
   unsigned long long timeout_ns;
 };
 
@@ -59,7 +63,8 @@ __device__ __forceinline__ void bulk_wait_all() {
 // CTAs per SM by register need: four (<= 64 registers) for W <= 4, three
 // for W = 5, two beyond.
 template <int W>
-constexpr int decode_ctas_per_sm() { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
+__host__ __device__ constexpr int decode_ctas_per_sm() { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
+inline int decode_ctas_per_sm(int W) { return W <= 4 ? 4 : (W == 5 ? 3 : 2); }
 
 template <int W, int D, bool MX, bool LV>
 __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
@@ -106,7 +111,59 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     *abort = 0;
     mbar_init_fence();
   }
-  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  const int row_part = (W - 1) * row_bytes;  // the state part of a stage
+  // sequences whose state rows are requested before the dependency wait
+  // (at most one per ring stage: sequence q < NS goes to stage q; none in
+  // the withheld-copy test mode, whose stages all take the normal path)
+  const int n_pre = (W > 1 && Gm.state_early && !Gm.withhold_first)
+                        ? min(min(nq, NS), SCONV_DECODE_EARLY_STAGES)
+                        : 0;
+  int issued0 = 0;  // (thread 0) stages already issued in full by the early fetch
+  if (Gm.state_early) {
+    // The caller promises that the previous kernel in the stream writes
+    // none of this call's inputs but k and v: thread 0 requests the state
+    // rows of the CTA's first n_pre sequences at once, waits for that
+    // kernel, and then requests their K/V rows -- so every stage it has
+    // started is complete (all its copies issued) before any wait that can
+    // give up, and the drain below sees every copy in flight.
+    if (threadIdx.x == 0) {
+      unsigned ok = 0;  // bit q: sequence q's state index is valid
+      for (int q = 0; q < n_pre; ++q) {
+        const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
+        const int64_t si = P.state_indices ? static_cast<int64_t>(P.state_indices[b]) : b;
+        if (si < 0 || si >= P.pool || (state_pos && state_pos[b] < 0)) continue;
+        ok |= 1u << q;
+        mbar_arrive_expect_tx(&full[q], static_cast<uint32_t>(stage_bytes));
+        unsigned char* dst = ring + static_cast<size_t>(q) * stage_bytes;
+        const uint16_t* sp = P.state + si * (W - 1) * srow;
+        if (full_slice) {
+          bulk_g2s(dst, sp, row_part, &full[q]);
+        } else {
+          for (int r = 0; r < W - 1; ++r) {
+            if (kn) bulk_g2s(dst + r * row_bytes, sp + r * srow + g0 * 8, kn * 16, &full[q]);
+            if (vn)
+              bulk_g2s(dst + r * row_bytes + kn * 16, sp + r * srow + P.C + (vg0 - half) * 8,
+                       vn * 16, &full[q]);
+          }
+        }
+      }
+      grid_dependency_wait();
+      for (int q = 0; q < n_pre; ++q) {
+        if (!(ok & (1u << q))) {
+          mbar_arrive(&full[q]);  // skipped sequence: an empty phase
+          continue;
+        }
+        const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
+        unsigned char* xd = ring + static_cast<size_t>(q) * stage_bytes + row_part;
+        if (kn) bulk_g2s(xd, P.k + b * P.row_stride + g0 * 8, kn * 16, &full[q]);
+        if (vn)
+          bulk_g2s(xd + kn * 16, P.v + b * P.row_stride + (vg0 - half) * 8, vn * 16, &full[q]);
+      }
+      issued0 = n_pre;
+    }
+  } else {
+    grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  }
   for (int q = threadIdx.x; q < nq; q += blockDim.x) {
     const int64_t b = b0 + static_cast<int64_t>(q) * Gm.ctas;
     int64_t si = b;
@@ -176,7 +233,7 @@ __global__ void __launch_bounds__(256, decode_ctas_per_sm<W>())
     }
     bulk_commit();
   };
-  int issued = 0;
+  int issued = issued0;
   auto drain = [&]() {  // after giving up: let issued loads land (bounded)
     for (int d = max(0, issued - NS); d < issued; ++d) {
       if (d == 0 && Gm.withhold_first) continue;  // never requested

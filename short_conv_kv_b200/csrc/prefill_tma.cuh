@@ -58,6 +58,11 @@ namespace sconv {
 #ifndef SCONV_PREFILL_MX_UNROLL
 #define SCONV_PREFILL_MX_UNROLL 2  // fast-path unroll of the MXFP8 store for W <= 4
 #endif
+#ifndef SCONV_PREFILL_FIRST_FILL
+// Chunks requested before the first one has landed (0 = the whole ring);
+// the rest of the ring is requested once chunk 0 has landed.
+#define SCONV_PREFILL_FIRST_FILL 0
+#endif
 #ifndef SCONV_PREFILL_BLOCK_LAYOUT
 // Stage layout: 1 = [K rows][V rows] (one bulk copy per part when rows are
 // packed), 0 = row by row (one copy per row part), 2 = per instance as
@@ -102,6 +107,7 @@ struct TmaGeom {
   int cut_r;      // num_tokens % ctas (the first cut_r ranges take one more token)
   int cu_smem;    // cu_seqlens copied to shared memory (num_seqs < kTmaCuSmemMax)
   int smem_ring;  // bytes of the stage ring
+  int state_wait_only;  // only conv_state reads wait for the previous kernel
   unsigned long long timeout_ns;
 };
 
@@ -177,9 +183,8 @@ __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 
   }
 }
 
-template <int W, int D, int MINB, bool MX, bool LV>
-__global__ void __launch_bounds__(kTmaMaxGroups, MINB)
-    prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
+template <int W, int D, bool MX, bool LV>
+__device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom& Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int R = kTmaRows;
   // layout variants (per-head gamma stride, ring-buffer state) only in the
@@ -190,6 +195,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
   const int S = P.num_seqs;
   const int T = static_cast<int>(P.num_tokens);
   const int NS = Gm.stages;
+  const int first_fill = SCONV_PREFILL_FIRST_FILL > 0 ? min(NS, SCONV_PREFILL_FIRST_FILL) : NS;
 
   // ---- channel slice of this CTA
   const int half = P.NG >> 1;
@@ -283,12 +289,22 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     *abort = 0;
     mbar_init_fence();
   }
-  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  // inputs may come from the previous kernel in the stream; with the
+  // state-only dependency only the reads of conv_state rows wait for it
+  if (!Gm.state_wait_only) grid_dependency_wait();
+  // This grid lets the next one launch (griddepcontrol.launch_dependents)
+  // once its copies are all issued; a CTA that has not waited for the
+  // previous grid yet does so first, so that the next grid never runs
+  // ahead of this grid's own predecessor.
+  auto trigger = [&]() {
+    if (Gm.state_wait_only) grid_dependency_wait();
+    allow_dependent_launch();
+  };
   if (kBlock && threadIdx.x == 0) {
     // full chunks that lie inside the even range: requested at once (block
     // layout only; in the W=4 bf16 instance the extra live values spill at
     // its 128-register cap, so it requests after the cut)
-    const int spec = S == 1 ? min(NS, (tb - first_row) / R) : 0;
+    const int spec = S == 1 ? min(first_fill, (tb - first_row) / R) : 0;
     for (; issued < spec; ++issued) issue(issued, issued);
   }
   if (Gm.cu_smem)
@@ -382,8 +398,8 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
   };
   if (threadIdx.x == 0) {
-    for (; issued < min(NS, nchunks); ++issued) issue(issued, issued);
-    if (issued == nchunks) allow_dependent_launch();
+    for (; issued < min(first_fill, nchunks); ++issued) issue(issued, issued);
+    if (issued == nchunks) trigger();
   }
 
   // =================================================================== consumers
@@ -466,6 +482,8 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     skip = !check_sequence(i, si);
     if (skip) return;
     if constexpr (W > 1) {
+      // the previous kernel in the stream may have written this state row
+      if (Gm.state_wait_only) grid_dependency_wait();
       const int a = cu(i), e = cu(i + 1);
       uint16_t* st = P.state + si * (W - 1) * srow + st_chan;
       // ring state: position p in row p mod (W-1); the window's oldest row
@@ -568,6 +586,11 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       if (threadIdx.x == 0) drain();
       return;
     }
+    if (SCONV_PREFILL_FIRST_FILL > 0 && c == 0 && threadIdx.x == 0 && issued < min(NS, nchunks)) {
+      // chunk 0 has landed: the rest of the ring
+      for (; issued < min(NS, nchunks); ++issued) issue(issued, issued);
+      if (issued == nchunks) trigger();
+    }
     const int r0 = first_row + c * R;
     const int rows = min(R, tb - r0);
     if (c % (SW / R) == 0) {
@@ -636,7 +659,7 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
       const uint32_t pp = s == 0 ? ph ^ 1u : ph;
       if (mbar_wait(&empty[sp], pp, abort, Gm.timeout_ns)) {
         issue(issued++, sp);
-        if (issued == nchunks) allow_dependent_launch();
+        if (issued == nchunks) trigger();
       } else {
         gave_up = true;
       }
@@ -652,6 +675,16 @@ __global__ void __launch_bounds__(kTmaMaxGroups, MINB)
     }
   }
 #undef NORM_STORE
+}
+
+template <int W, int D, int MINB, bool MX, bool LV>
+__global__ void __launch_bounds__(kTmaMaxGroups, MINB)
+    prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
+  prefill_body<W, D, MX, LV>(P, Gm);
+  // With the state-only dependency a CTA that never touched a state row has
+  // not waited for the previous grid yet: it does before it exits, so this
+  // grid's completion still implies its predecessor's.
+  if (Gm.state_wait_only && threadIdx.x == 0) grid_dependency_wait();
 }
 
 }  // namespace sconv

@@ -9,8 +9,7 @@
 
 #include "sconv_kv.h"
 #include "common.cuh"
-#include "decode_tma.cuh"
-#include "prefill_tma.cuh"
+#include "instances.h"
 #include "stages.cuh"
 
 namespace {
@@ -22,74 +21,19 @@ thread_local char g_cuda_error[256] = "";
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-using TmaFn = void (*)(StepParams, sconv::TmaGeom);
+using sconv::TmaFn;
+using sconv::DecFn;
 
-// W <= 4 fits 128 registers: two CTAs per SM (twice the warps to hide
-// latency); wider windows need more registers and run one CTA per SM.
-template <int W>
-constexpr int prefill_ctas_per_sm() { return W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1; }
-
-using DecFn = void (*)(StepParams, sconv::DecGeom);
-
-// Kernel instance for (W, D): F<W, D>() over W in 1..8, D in {64, 128, 256}.
-template <typename Fn, template <int, int> class F>
-struct Pick {
-  template <int D>
-  static Fn by_w(int W) {
-    switch (W) {
-      case 1: return F<1, D>::get();
-      case 2: return F<2, D>::get();
-      case 3: return F<3, D>::get();
-      case 4: return F<4, D>::get();
-      case 5: return F<5, D>::get();
-      case 6: return F<6, D>::get();
-      case 7: return F<7, D>::get();
-      case 8: return F<8, D>::get();
-      default: return nullptr;
-    }
-  }
-  static Fn get(int W, int D) {
-    switch (D) {
-      case 64: return by_w<64>(W);
-      case 128: return by_w<128>(W);
-      case 256: return by_w<256>(W);
-      default: return nullptr;
-    }
-  }
-};
-// Kernel instances: bf16 or MXFP8 store (MX), without or with the layout
-// variants (LV: per-head gamma stride, ring-buffer state).
-template <bool MX, bool LV>
-struct DecodeKs {
-  template <int W, int D>
-  struct K {
-    static DecFn get() { return sconv::decode_tma_kernel<W, D, MX, LV>; }
-  };
-};
-template <bool MX, bool LV>
-struct PrefillKs {
-  template <int W, int D>
-  struct K {
-    static TmaFn get() {
-      return sconv::prefill_tma_kernel<W, D, prefill_ctas_per_sm<W>(), MX, LV>;
-    }
-  };
-};
 bool uses_layout_variants(const sconv_kv_options_t* opts) {
   return opts && (opts->gamma_head_stride != 0 || opts->state_positions != nullptr);
 }
+// Kernel instances live in their own translation units (compiled in
+// parallel): bf16 or MXFP8 store, without or with the layout variants.
 TmaFn pick_prefill(int W, int D, bool mx, bool lv) {
-  if (mx) return lv ? Pick<TmaFn, PrefillKs<true, true>::K>::get(W, D)
-                    : Pick<TmaFn, PrefillKs<true, false>::K>::get(W, D);
-  return lv ? Pick<TmaFn, PrefillKs<false, true>::K>::get(W, D)
-            : Pick<TmaFn, PrefillKs<false, false>::K>::get(W, D);
+  if (mx) return lv ? sconv::pick_prefill_mx_lv(W, D) : sconv::pick_prefill_mx(W, D);
+  return lv ? sconv::pick_prefill_bf16_lv(W, D) : sconv::pick_prefill_bf16(W, D);
 }
-DecFn pick_decode(int W, int D, bool mx, bool lv) {
-  if (mx) return lv ? Pick<DecFn, DecodeKs<true, true>::K>::get(W, D)
-                    : Pick<DecFn, DecodeKs<true, false>::K>::get(W, D);
-  return lv ? Pick<DecFn, DecodeKs<false, true>::K>::get(W, D)
-            : Pick<DecFn, DecodeKs<false, false>::K>::get(W, D);
-}
+DecFn pick_decode(int W, int D, bool mx, bool lv) { return sconv::pick_decode(W, D, mx, lv); }
 
 // Host-side caches (SM counts, shared-memory attributes, scratch addresses)
 // are shared by every host thread that calls the library.
@@ -356,7 +300,7 @@ int prefill_impl(
   G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
   const int stage_bytes = sconv::kTmaRows * G.slice * 16;
-  const int per_sm = W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1;  // = prefill_ctas_per_sm<W>()
+  const int per_sm = sconv::prefill_ctas_per_sm(W);
   int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
   // + per-warp slot-offset tables + per-thread gammas
@@ -374,6 +318,7 @@ int prefill_impl(
                      ? static_cast<unsigned long long>(opts->wait_timeout_ns)
                      : 1000000000ull;
   G.withhold_first = (opts && opts->withhold_first_copy) ? 1 : 0;
+  G.state_wait_only = (opts && opts->state_only_dependency) ? 1 : 0;
   const size_t smem = smem_base + (G.cu_smem ? cu_bytes : 0);
   if (!smem_attr_set(reinterpret_cast<const void*>(fn), smem)) {
     snprintf(g_cuda_error, sizeof g_cuda_error, "cudaFuncSetAttribute failed");
@@ -433,7 +378,7 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
   G.slice = P.NG < 256 ? P.NG : 256;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
   const int stage_bytes = W * G.slice * 16;
-  const int per_sm = W <= 4 ? 4 : (W == 5 ? 3 : 2);  // = decode_ctas_per_sm<W>()
+  const int per_sm = sconv::decode_ctas_per_sm(W);
   int stages = (192 * 1024 / per_sm) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
   G.smem_ring = G.stages * stage_bytes;
@@ -441,6 +386,7 @@ int decode_impl(const void* k, const void* v, int64_t row_stride, int batch,
                      ? static_cast<unsigned long long>(opts->wait_timeout_ns)
                      : 1000000000ull;
   G.withhold_first = (opts && opts->withhold_first_copy) ? 1 : 0;
+  G.state_early = (opts && opts->independent_state) ? 1 : 0;
   int64_t ctas = static_cast<int64_t>(sm_count()) * per_sm / ctas_y;
   const int64_t need = (static_cast<int64_t>(batch) + sconv::kDecMaxSeqs - 1) / sconv::kDecMaxSeqs;
   if (ctas < need) ctas = need;

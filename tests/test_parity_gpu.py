@@ -114,6 +114,20 @@ def test_varlen_32_sequences_sampled():
     _check_sampled(b, kc, vc, st, tokens)
 
 
+def test_many_sequences_1900_sampled():
+    """1,900 sequences of 32..96 tokens, Hkv=8, D=128, W=4: cu_seqlens no
+    longer fits in shared memory beside two CTAs per SM, so the CTAs read it
+    from global memory (and all stay resident); sampled tokens of every
+    sequence start, the full state, untouched slots against the oracle."""
+    g = torch.Generator().manual_seed(3600)
+    lengths = torch.randint(32, 97, (1900,), generator=g).tolist()
+    b = wl.make_prefill(lengths, Hkv=8, D=128, W=4, seed=3601, state="normal",
+                        page_size=64, permute_pages=True, spare_pages=64)
+    kc, vc, st = gu.run_gpu_prefill(b)
+    tokens = _sample_tokens(b.cu_seqlens.numpy(), b.W, np.random.default_rng(19), n_random=500)
+    _check_sampled(b, kc, vc, st, tokens)
+
+
 def test_varlen_subset_full():
     """Whole-batch oracle on 6 of the varlen workload's sequences (packed as
     their own batch with their own initial state rows)."""
@@ -185,6 +199,86 @@ def test_long_context_1m_chunked_sampled():
         assert np.array_equal(wl.bits(st.cpu()), prev_tail), f"state after chunk {c}"
         all_slots.append(sm)
     _check_untouched_device(kc, vc, torch.cat(all_slots))
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+def test_chunks_back_to_back_sampled(overlap):
+    """Six 65,536-token chunks of one sequence launched back to back on one
+    stream with no synchronisation in between -- with the state-only
+    dependency (only the CTA that reads the carried state waits for the
+    previous launch) and without it.  Afterwards: sampled tokens of every
+    chunk (incl. each chunk's first W-1, whose window reaches into the
+    previous chunk, and every chunk's last rows) against the oracle, the
+    final state bit for bit, untouched slots."""
+    b = _binding()
+    s = wl.long_context(seed=5300)
+    n = 6
+    C, W = s.C, s.W
+    chunks = [s.chunk_inputs(c) for c in range(n)]
+    dev_chunks = [tuple(gu.dev(x) for x in ch) for ch in chunks]
+    st = gu.dev(s.initial_state())
+    kc, vc = gu.dev(s.empty_cache()), gu.dev(s.empty_cache())
+    wk, wv, gk, gv = (gu.dev(s.conv_w_k), gu.dev(s.conv_w_v), gu.dev(s.gamma_k),
+                      gu.dev(s.gamma_v))
+    torch.cuda.synchronize()
+    for k, v, sm, cu in dev_chunks:
+        b.prefill_varlen(k, v, cu, wk, wv, gk, gv, s.eps, st, sm, kc, vc,
+                         state_only_dependency=overlap)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(53)
+    prev_tail = wl.bits(s.initial_state())
+    for c, (k, v, sm, cu) in enumerate(chunks):
+        L = k.shape[0]
+        kb, vb = wl.bits(k).reshape(L, C), wl.bits(v).reshape(L, C)
+        tokens = _sample_tokens(np.array([0, L]), W, rng, n_random=150)
+        zk, zv = gu.sampled_oracle_z(kb, vb, np.array([0, L]), prev_tail, tokens, W,
+                                     wl.bits(s.conv_w_k), wl.bits(s.conv_w_v),
+                                     s.gamma_k.numpy(), s.gamma_v.numpy(), s.eps, s.Hkv, s.D)
+        slots = gu.dev(sm[tokens])
+        gu.assert_close(wl.bits(kc.reshape(-1, C)[slots].cpu()), zk, f"k chunk {c}")
+        gu.assert_close(wl.bits(vc.reshape(-1, C)[slots].cpu()), zv, f"v chunk {c}")
+        prev_tail = gu.expected_final_state(kb, vb, np.array([0, L]), prev_tail, W)
+    assert np.array_equal(wl.bits(st.cpu()), prev_tail), "state after the chain"
+    _check_untouched_device(kc, vc, torch.cat([ch[2] for ch in chunks]))
+
+
+def test_varlen_chunks_back_to_back_state_only_dependency():
+    """Four continuation chunks of the same 8 sequences (state carried in a
+    shuffled pool), launched back to back with the state-only dependency:
+    here most CTAs hold a sequence start and wait; the rest stream at once.
+    Each chunk against the oracle run on the state the previous chunk left."""
+    b = _binding()
+    n_seq, pool = 8, 11
+    si = torch.tensor([3, 10, 0, 7, 5, 9, 1, 2], dtype=torch.int32)
+    batches = [wl.make_prefill(list(np.random.default_rng(60 + c).integers(0, 700, n_seq)),
+                               Hkv=4, D=128, W=4, seed=6100 + c, state="normal",
+                               page_size=16, spare_pages=0, pool_size=pool,
+                               state_indices=si) for c in range(4)]
+    st0 = batches[0].conv_state.clone()
+    st = gu.dev(st0)
+    caches = [(gu.dev(x.empty_cache()), gu.dev(x.empty_cache())) for x in batches]
+    w = [gu.dev(t) for t in (batches[0].conv_w_k, batches[0].conv_w_v, batches[0].gamma_k,
+                             batches[0].gamma_v)]
+    devs = [(gu.dev(x.k), gu.dev(x.v), gu.dev(x.cu_seqlens), gu.dev(x.slot_mapping))
+            for x in batches]
+    sid = gu.dev(si)
+    torch.cuda.synchronize()
+    for (k, v, cu, sm), (kc, vc) in zip(devs, caches):
+        b.prefill_varlen(k, v, cu, *w, batches[0].eps, st, sm, kc, vc, state_indices=sid,
+                         state_only_dependency=True)
+    torch.cuda.synchronize()
+    state = wl.bits(st0)
+    for c, (x, (kc, vc)) in enumerate(zip(batches, caches)):
+        x.conv_w_k, x.conv_w_v = batches[0].conv_w_k, batches[0].conv_w_v
+        x.gamma_k, x.gamma_v = batches[0].gamma_k, batches[0].gamma_v
+        x.conv_state = wl.from_bits(state)
+        ref = gu.oracle_prefill(x)
+        gu.check_cache(wl.bits(kc.cpu()), ref["k_cache"], x.slot_mapping.numpy(), ref["z_k"],
+                       f"k chunk {c}")
+        gu.check_cache(wl.bits(vc.cpu()), ref["v_cache"], x.slot_mapping.numpy(), ref["z_v"],
+                       f"v chunk {c}")
+        state = ref["conv_state"]
+    assert np.array_equal(wl.bits(st.cpu()), state)
 
 
 @pytest.mark.parametrize("W", [2, 4, 8])
@@ -440,3 +534,54 @@ def test_skewed_lengths_full():
     b = wl.make_prefill(lengths, Hkv=4, D=128, W=4, seed=905, state="normal",
                         page_size=16, spare_pages=4)
     gu.full_parity(b)
+
+
+@pytest.mark.parametrize("ring", [False, True])
+def test_decode_independent_state_alternating_batches(ring):
+    """Two decode batches with disjoint state rows in one pool, launched
+    alternately with the independent-state promise (each call's previous
+    kernel is the other batch's step, which writes none of this call's
+    state rows), 8 steps each with no synchronisation in between.  Every
+    step's cache rows and the final states against two oracle chains."""
+    import oracle
+    b = _binding()
+    B, steps = 256, 8
+    sA = wl.decode(seed=7100, batch=B, pages_per_seq=1, page_size=16, max_start=8)
+    sB = wl.decode(seed=7200, batch=B, pages_per_seq=1, page_size=16, max_start=8)
+    C = sA.C
+    pool = torch.cat([sA.conv_state, sB.conv_state])
+    st = gu.dev(pool.clone())
+    idx = [gu.dev(torch.arange(B, dtype=torch.int32)),
+           gu.dev(torch.arange(B, 2 * B, dtype=torch.int32))]
+    setups = [sA, sB]
+    w = [gu.dev(x) for x in (sA.conv_w_k, sA.conv_w_v, sA.gamma_k, sA.gamma_v)]
+    caches = [(gu.dev(s.empty_cache()), gu.dev(s.empty_cache())) for s in setups]
+    inputs = [[s.step_inputs(t) for t in range(steps)] for s in setups]
+    dev_in = [[tuple(gu.dev(x) for x in inp) for inp in seq] for seq in inputs]
+    pos = [[gu.dev(torch.from_numpy(s.start_len.astype(np.int64) + t)) for t in range(steps)]
+           for s in setups]
+    torch.cuda.synchronize()
+    for t in range(steps):
+        for j in range(2):
+            k, v, sm = dev_in[j][t]
+            b.decode(k, v, *w, sA.eps, st, sm, *caches[j], state_indices=idx[j],
+                     state_positions=pos[j][t] if ring else None, independent_state=True)
+    torch.cuda.synchronize()
+    small = np.zeros((B, 1, sA.Hkv, sA.D), np.uint16)
+    for j, s in enumerate(setups):
+        ref_state = wl.bits(s.conv_state)
+        kc, vc = caches[j]
+        for t in range(steps):
+            k, v, sm = inputs[j][t]
+            ref = oracle.decode(wl.bits(k), wl.bits(v), wl.bits(sA.conv_w_k),
+                                wl.bits(sA.conv_w_v), sA.gamma_k.numpy(), sA.gamma_v.numpy(),
+                                sA.eps, ref_state, np.arange(B, dtype=np.int64), small,
+                                small.copy(),
+                                state_positions=(s.start_len.astype(np.int64) + t) if ring
+                                else None)
+            ref_state = ref["conv_state"]
+            slots = gu.dev(sm)
+            gu.assert_close(wl.bits(kc.reshape(-1, C)[slots].cpu()), ref["z_k"], f"k {j} {t}")
+            gu.assert_close(wl.bits(vc.reshape(-1, C)[slots].cpu()), ref["z_v"], f"v {j} {t}")
+        got = wl.bits(st.cpu())[j * B:(j + 1) * B]
+        assert np.array_equal(got, ref_state), f"state of batch {j}"

@@ -49,7 +49,10 @@ def test_prefill_wait_timeout_sets_flag_and_context_survives():
                                    page_size=16, spare_pages=1))
 
 
-def test_decode_wait_timeout_sets_flag_and_context_survives():
+@pytest.mark.parametrize("early", [False, True])
+def test_decode_wait_timeout_sets_flag_and_context_survives(early):
+    """(early: with the independent-state promise, whose CTAs request their
+    state rows before the dependency wait.)"""
     from short_conv_kv_b200 import binding as bd
     s = wl.decode(seed=2910)
     k, v, sm = s.step_inputs(0)
@@ -60,7 +63,7 @@ def test_decode_wait_timeout_sets_flag_and_context_survives():
         kc, vc = gu.dev(s.empty_cache()), gu.dev(s.empty_cache())
         st = gu.dev(s.conv_state.clone())
         bd.decode(k, v, *w, s.eps, st, sm, kc, vc, err_flag=err, wait_timeout_ns=100_000,
-                  withhold_first_copy=True)
+                  withhold_first_copy=True, independent_state=early)
 
     assert _timed_out(call)
     # a normal decode step right after: state bit-exact, no flag
