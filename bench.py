@@ -188,6 +188,10 @@ class Workload:
     same algorithmic bytes (`bytes_per_launch`)."""
 
     def __init__(self, name, rank):
+        # decode calls with the independent-state promise (the previous
+        # launch writes none of a call's state rows)
+        self.early_state = name.endswith("_early")
+        name = name[:-6] if self.early_state else name
         self.mx = name.endswith("_mx")  # MXFP8 cache store variant
         name = name[:-3] if self.mx else name
         self.ring = name.endswith("_ring")  # ring-buffer conv_state (decode)
@@ -196,9 +200,6 @@ class Workload:
         # prefill calls with the state-only dependency (the previous launch
         # writes none of a call's inputs but conv_state): set by the caller
         self.chain_overlap = False
-        # decode calls with the independent-state promise (the previous
-        # launch writes none of a call's state rows): set by the caller
-        self.early_state = False
         seed_shift = 97 * rank
         if name == "single":
             self.kind, self.batches = "prefill", [wl.single(seed=2000 + seed_shift)]
@@ -243,6 +244,8 @@ class Workload:
             self.desc = "decode 1024 seqs x 1 token, Hkv=8, D=128, W=4, N(0,1) state, 4096-page cache"
             if name == "decode_ring":
                 self.desc += "; ring-buffer state (one state row written per sequence)"
+            if self.early_state:
+                self.desc += "; independent-state promise (state rows requested before the wait)"
         else:
             raise SystemExit(f"unknown workload {name}")
 
@@ -628,6 +631,8 @@ SIDE_CONFIGS = [
     ("single", "single-sequence prefill T=8192"),
     ("varlen", "varlen prefill, 32 sequences"),
     ("decode", "decode step, 1024 sequences"),
+    ("decode_early", "decode step, 1024 sequences, calls with the independent-state promise "
+                     "(the launch before each writes none of its state rows)"),
     ("wsweep2", "65,536-token prefill, W=2"),
     ("wsweep8", "65,536-token prefill, W=8"),
 ]
@@ -636,8 +641,9 @@ SIDE_MAX_LAUNCHES = 2500
 
 
 def time_isolated_launch(work, dev, reps=7):
-    """Median time of one launch on an idle GPU (synchronised before and
-    after, CUDA events around the single launch): the time a call takes
+    """Median time of one launch with nothing before or after it on the GPU
+    (a sleep kernel ahead of the start event hides the host's launch
+    latency; CUDA events around the single launch): the time a call takes
     when nothing overlaps it, set against the chain's time per launch."""
     stream = torch.cuda.Stream(device=dev)
     times = []
@@ -645,6 +651,8 @@ def time_isolated_launch(work, dev, reps=7):
         call = work.prepared(i, stream)
         s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(SLEEP_CYCLES // 20)  # ~0.1 ms
         s_ev.record(stream)
         call()
         e_ev.record(stream)
@@ -704,7 +712,7 @@ def run_ours(args):
     # dependency is for: the long-context workload promises it by default
     work.chain_overlap = work.kind != "decode" and (
         args.chain_overlap or (work.kind == "long" and not args.no_chain_overlap))
-    work.early_state = args.early_state and work.kind == "decode"
+    work.early_state = (work.early_state or args.early_state) and work.kind == "decode"
     work.setup(dev)
     K, Wu = args.steps, args.warmup
     lps = work.launches_per_step
@@ -896,7 +904,8 @@ def main():
                     choices=["long", "single", "varlen", "skew", "decode", "decode_ring", "wsweep2",
                              "wsweep4", "wsweep8", "many",
                              "single_mx", "varlen_mx", "decode_mx", "long_mx", "wsweep2_mx",
-                             "wsweep4_mx", "wsweep8_mx"])
+                             "wsweep4_mx", "wsweep8_mx", "decode_early", "decode_mx_early",
+                             "decode_ring_early"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true",

@@ -151,7 +151,10 @@ SCONV_KV_API int sconv_kv_cache_layout(int64_t num_pages, int64_t page_size,
  *                 means "do not write" (padding).
  *  k_cache, v_cache  bf16 caches described by *layout (host pointer to the
  *                 struct).  16-byte aligned; stride_head, stride_slot and
- *                 stride_page multiples of 8 elements.
+ *                 stride_page multiples of 8 elements; the element offset
+ *                 of the last slot's row, (num_pages-1)*stride_page +
+ *                 (page_size-1)*stride_slot, below 8 * (2^32 - 1) (about
+ *                 34 G elements; SCONV_KV_ERR_SHAPE otherwise).
  *  err_flag       optional device int; SCONV_KV_FLAG_* bits are OR-ed in.
  *  stream         cudaStream_t as void*.
  *

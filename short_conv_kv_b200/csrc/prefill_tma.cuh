@@ -94,7 +94,16 @@ __host__ __device__ constexpr bool block_layout() {
 }
 constexpr int kTmaRingBytes2 = SCONV_PREFILL_RING_KB * 1024;
 constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memory
-constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 8;  // per-warp slot offsets
+// per-warp slot tables: the cache row offset of each row of a 32-row window
+// in units of 8 elements (kNoRow: not written), 4 bytes per row; the host
+// refuses caches whose row offsets do not fit
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 4;
+// Every stage is laid out for a full slice: R rows of kTmaMaxGroups * 16
+// bytes (the row layout keeps that fixed pitch between rows, so a thread's
+// per-token shared-memory loads take immediate offsets).
+constexpr int kTmaRowPitch = kTmaMaxGroups * 16;
+constexpr int kTmaStageBytes = kTmaRows * kTmaRowPitch;
 constexpr int kTmaGammaBytes = kTmaMaxGroups * 32;  // 8 gammas per thread (W <= 4)
 
 struct TmaGeom {
@@ -216,8 +225,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
   int* s_cu = const_cast<int*>(reinterpret_cast<volatile int*>(empty + NS) + 12);
   // per-warp table of the cache row offsets of the current 32-row window
   // (host reserves 8 warps x 32 x 8 bytes right below the barriers)
-  long long* warp_off =
-      reinterpret_cast<long long*>(smem + Gm.smem_ring - kTmaOffTableBytes) + (threadIdx.x >> 5) * 32;
+  uint32_t* warp_off =
+      reinterpret_cast<uint32_t*>(smem + Gm.smem_ring - kTmaOffTableBytes) + (threadIdx.x >> 5) * 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -247,7 +256,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
     const int r0 = first_row + c * R;
     const int rows = min(R, tb - r0);
     mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(rows * row_bytes));
-    unsigned char* sdst = ring + static_cast<size_t>(st) * R * row_bytes;
+    unsigned char* sdst = ring + static_cast<size_t>(st) * kTmaStageBytes;
     const uint16_t* ksrc = P.k + static_cast<int64_t>(r0) * P.row_stride + g0 * 8;
     const uint16_t* vsrc = P.v + static_cast<int64_t>(r0) * P.row_stride + (vg0 - half) * 8;
     if constexpr (kBlock) {
@@ -275,7 +284,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
         const int64_t o = static_cast<int64_t>(r) * P.row_stride;
         if (kn) bulk_g2s(sdst, ksrc + o, kn * 16, &full[st]);
         if (vn) bulk_g2s(sdst + kn * 16, vsrc + o, vn * 16, &full[st]);
-        sdst += row_bytes;
+        sdst += kTmaRowPitch;
       }
     }
   };
@@ -548,16 +557,19 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
   }
 
   const float eps = P.eps, inv_d = P.inv_d;
+  // `off8`: the row's cache offset in units of 8 elements (bf16: 16 bytes;
+  // MXFP8: 8 code bytes, and a quarter of a scale byte), kNoRow if unwritten
 #define NORM_STORE(pred)                                                            \
   do {                                                                              \
-    uint8_t* mxd = MX ? mxdata + off : nullptr;                                     \
-    uint8_t* mxs = MX ? mxscale + (off >> 5) : nullptr;                             \
+    uint8_t* mxd = MX ? mxdata + static_cast<uint64_t>(off8) * 8 : nullptr;         \
+    uint8_t* mxs = MX ? mxscale + (off8 >> 2) : nullptr;                            \
+    uint16_t* cdst = MX ? nullptr : cache + static_cast<uint64_t>(off8) * 8;        \
     if constexpr (gamma_in_smem<W>()) {                                             \
       float2 gs[4];                                                                 \
       lds_gamma(my_gamma, gs);                                                      \
-      norm_store<D, MX>(acc, gs, inv_d, eps, (pred), cache + off, mxd, mxs);        \
+      norm_store<D, MX>(acc, gs, inv_d, eps, (pred), cdst, mxd, mxs);               \
     } else {                                                                        \
-      norm_store<D, MX>(acc, gm, inv_d, eps, (pred), cache + off, mxd, mxs);        \
+      norm_store<D, MX>(acc, gm, inv_d, eps, (pred), cdst, mxd, mxs);               \
     }                                                                               \
   } while (0)
   // inactive lanes read column 0 (and never store): no predicated loads
@@ -565,7 +577,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
       !kBlock ? ring + (active ? lg : 0) * 16
               : ring + (!active ? 0 : lg < kn ? lg * 16 : R * kn * 16 + (lg - kn) * 16);
   // bytes between consecutive rows of this thread's part of a stage
-  const int my_rs = !kBlock ? row_bytes : (active && lg >= kn) ? vn * 16 : kn * 16;
+  const int my_rs = !kBlock ? kTmaRowPitch : (active && lg >= kn) ? vn * 16 : kn * 16;
   // slot_mapping is read one 32-row window ahead of use, lane l holding row
   // (window start + l), so its load latency hides behind four chunks.
   constexpr int SW = (32 / R) * R;
@@ -597,12 +609,15 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
       // rows [r0, r0 + SW): lane l writes row r0 + l's cache row offset
       // (-1, masked, for the rows of chunk 0 in front of ta)
       __syncwarp();
-      warp_off[lane] = (c == 0 && lane < *s_skip) ? -1 : slot_row_offset(P, next_slot, report_slots);
+      // (rows past the range's end have slot -1: their stores are masked
+      // here, so the fast path needs no row bound)
+      const int64_t ro = (c == 0 && lane < *s_skip) ? -1 : slot_row_offset(P, next_slot, report_slots);
+      warp_off[lane] = ro < 0 ? kNoRow : static_cast<uint32_t>(ro >> 3);
       __syncwarp();
       next_slot = load_slot(c / (SW / R) + 1);
     }
     const int sbase = (c % (SW / R)) * R;  // this chunk's first lane
-    const unsigned char* stage = my_ring + static_cast<size_t>(s) * R * row_bytes;
+    const unsigned char* stage = my_ring + static_cast<size_t>(s) * kTmaStageBytes;
     if (next >= r0 + rows && !skip) {
       // fast path: up to R tokens of one sequence, no branches (rows past
       // the end of the range compute on stale data and are not stored).
@@ -619,8 +634,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
             const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
             float2 acc[4];
             conv_step<W>(tw, win, xr, acc);
-            const long long off = warp_off[sbase + r];
-            NORM_STORE(active && r < rows && off >= 0);
+            const uint32_t off8 = warp_off[sbase + r];
+            NORM_STORE(active && off8 != kNoRow);
           }
         }
       } else {
@@ -629,8 +644,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
           const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
           float2 acc[4];
           conv_step<W>(tw, win, xr, acc);
-          const long long off = warp_off[sbase + r];
-          NORM_STORE(active && r < rows && off >= 0);
+          const uint32_t off8 = warp_off[sbase + r];
+          NORM_STORE(active && off8 != kNoRow);
         }
       }
     } else {
@@ -645,8 +660,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
         float2 acc[4];
         conv_step<W>(tw, win, xr, acc);
-        const long long off = warp_off[sbase + r];
-        NORM_STORE(active && !skip && off >= 0);
+        const uint32_t off8 = warp_off[sbase + r];
+        NORM_STORE(active && !skip && off8 != kNoRow);
       }
     }
     __syncwarp();

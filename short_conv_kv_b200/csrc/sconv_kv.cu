@@ -283,6 +283,14 @@ int prefill_impl(
   if (!cu_seqlens) return SCONV_KV_ERR_NULL;
   TmaFn fn = pick_prefill(W, head_dim, mx, uses_layout_variants(opts));
   if (!fn) return SCONV_KV_ERR_UNSUPPORTED;
+  // the kernel keeps cache row offsets in 32 bits, in units of 8 elements
+  {
+    const __int128 last_row =
+        static_cast<__int128>(layout->num_pages > 0 ? layout->num_pages - 1 : 0) *
+            layout->stride_page +
+        static_cast<__int128>(layout->page_size - 1) * layout->stride_slot;
+    if (last_row / 8 >= static_cast<__int128>(sconv::kNoRow)) return SCONV_KV_ERR_SHAPE;
+  }
 
   P.num_tokens = num_tokens;
   P.cu_seqlens = cu_seqlens;
@@ -299,7 +307,7 @@ int prefill_impl(
   sconv::TmaGeom G;
   G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
-  const int stage_bytes = sconv::kTmaRows * G.slice * 16;
+  const int stage_bytes = sconv::kTmaStageBytes;  // laid out for a full slice
   const int per_sm = sconv::prefill_ctas_per_sm(W);
   int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);

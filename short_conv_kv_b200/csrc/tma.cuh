@@ -58,14 +58,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns
-// false (and raises *abort) on timeout; returns false at once if *abort is
-// already raised by another thread.
+// false (and raises *abort) on timeout; returns false soon after another
+// thread has raised *abort.  The clock and the abort flag are checked once
+// per 8 polls (each poll may suspend the thread for a while in hardware),
+// so a waiting warp takes few issue slots from the warps that compute.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)  // unrolled: no counter register
+      if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (global_ns() - t0 > timeout_ns) {
       *abort = 1;
