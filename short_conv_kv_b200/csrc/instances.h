@@ -13,14 +13,13 @@ namespace sconv {
 using TmaFn = void (*)(StepParams, TmaGeom);
 using DecFn = void (*)(StepParams, DecGeom);
 
-// Persistent prefill CTAs per SM: W <= 4 fits 128 registers, two CTAs per
-// SM (twice the warps to hide latency); wider windows need more registers
-// and run one CTA per SM.
-template <int W>
-__host__ __device__ constexpr int prefill_ctas_per_sm() {
-  return W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1;
+// Persistent prefill CTAs per SM (prefill_ctas_per_sm<W, MX>() in
+// prefill_tma.cuh): W <= 4 fits 128 registers, two CTAs per SM (twice the
+// warps to hide latency); wider windows need more registers and run one CTA
+// per SM.
+inline int prefill_ctas_per_sm(int W, bool mx) {
+  return W <= 4 ? (mx ? SCONV_PREFILL_MX_PER_SM : SCONV_PREFILL_SMALL_W_PER_SM) : 1;
 }
-inline int prefill_ctas_per_sm(int W) { return W <= 4 ? SCONV_PREFILL_SMALL_W_PER_SM : 1; }
 
 // nullptr for an unsupported (W, D).
 TmaFn pick_prefill_bf16(int W, int D);

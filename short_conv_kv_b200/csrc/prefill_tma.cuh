@@ -56,7 +56,15 @@ namespace sconv {
 #define SCONV_PREFILL_BF16_UNROLL 4  // fast-path unroll of the bf16 store for W <= 4
 #endif
 #ifndef SCONV_PREFILL_MX_UNROLL
-#define SCONV_PREFILL_MX_UNROLL 2  // fast-path unroll of the MXFP8 store for W <= 4
+#define SCONV_PREFILL_MX_UNROLL 8  // fast-path unroll of the MXFP8 store for W <= 4
+#endif
+#ifndef SCONV_PREFILL_MX_PER_SM
+// CTAs per SM of the MXFP8 store for W <= 4.  Measured on B200: one CTA
+// per SM with an 8-token unroll and gammas in registers (211 registers)
+// against two with a 2-token unroll: 65,536-token launch 102.1 -> 91.9 us,
+// 8192-token launch 19.1 -> 18.0 us, varlen batch 220.5 -> 197.4 us (the
+// MX store's longer per-token chain needs the wider unroll).
+#define SCONV_PREFILL_MX_PER_SM 1
 #endif
 #ifndef SCONV_PREFILL_FIRST_FILL
 // Chunks requested before the first one has landed (0 = the whole ring);
@@ -77,8 +85,12 @@ constexpr int kTmaRows = SCONV_PREFILL_ROWS;  // token rows per stage
 // path is unrolled by 4 and gamma is read from shared memory per token,
 // which frees the registers the unrolled tokens need; wider windows run one
 // CTA per SM with room for an 8-token unroll and gamma in registers.
-template <int W>
-__host__ __device__ constexpr bool gamma_in_smem() { return W <= 4; }
+template <int W, bool MX>
+__host__ __device__ constexpr int prefill_ctas_per_sm() {
+  return W <= 4 ? (MX ? SCONV_PREFILL_MX_PER_SM : SCONV_PREFILL_SMALL_W_PER_SM) : 1;
+}
+template <int W, bool MX>
+__host__ __device__ constexpr bool gamma_in_smem() { return prefill_ctas_per_sm<W, MX>() > 1; }
 template <int W, bool MX>
 __host__ __device__ constexpr int fast_unroll() {
   return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : SCONV_PREFILL_BF16_UNROLL) : 8;
@@ -442,7 +454,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
     const float* gam = (isv ? P.gamma_v : P.gamma_k) + (c0 / D) * gamma_hs + d0;
     const float4 a = __ldg(reinterpret_cast<const float4*>(gam));
     const float4 b = __ldg(reinterpret_cast<const float4*>(gam) + 1);
-    if constexpr (gamma_in_smem<W>()) {
+    if constexpr (gamma_in_smem<W, MX>()) {
       reinterpret_cast<float4*>(my_gamma)[0] = a;
       reinterpret_cast<float4*>(my_gamma)[1] = b;
     } else {
@@ -564,7 +576,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
     uint8_t* mxd = MX ? mxdata + static_cast<uint64_t>(off8) * 8 : nullptr;         \
     uint8_t* mxs = MX ? mxscale + (off8 >> 2) : nullptr;                            \
     uint16_t* cdst = MX ? nullptr : cache + static_cast<uint64_t>(off8) * 8;        \
-    if constexpr (gamma_in_smem<W>()) {                                             \
+    if constexpr (gamma_in_smem<W, MX>()) {                                             \
       float2 gs[4];                                                                 \
       lds_gamma(my_gamma, gs);                                                      \
       norm_store<D, MX>(acc, gs, inv_d, eps, (pred), cdst, mxd, mxs);               \

@@ -308,7 +308,7 @@ int prefill_impl(
   G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
   const int stage_bytes = sconv::kTmaStageBytes;  // laid out for a full slice
-  const int per_sm = sconv::prefill_ctas_per_sm(W);
+  const int per_sm = sconv::prefill_ctas_per_sm(W, mx);
   int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
   // + per-warp slot-offset tables + per-thread gammas
