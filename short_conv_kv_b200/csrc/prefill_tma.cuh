@@ -16,7 +16,7 @@
 //
 // Pipeline.  The rows of the CTA's range (the W-1 rows in front of a range
 // that starts inside a sequence are read directly) stream through a ring of
-// `stages` shared-memory stages of kTmaRows token rows each, filled by bulk
+// `stages` shared-memory stages of R token rows each, filled by bulk
 // asynchronous copies (for packed rows, one per chunk for K and one for V;
 // otherwise one per row part), completion counted in bytes on the stage's
 // "full" barrier.  Every warp waits on "full", copies
@@ -79,7 +79,15 @@ namespace sconv {
 #endif
 
 constexpr int kTmaMaxGroups = 256;   // channel groups per CTA slice
-constexpr int kTmaRows = SCONV_PREFILL_ROWS;  // token rows per stage
+#ifndef SCONV_PREFILL_ROWS_SMALL_W
+#define SCONV_PREFILL_ROWS_SMALL_W SCONV_PREFILL_ROWS  // token rows per stage for W <= 4
+#endif
+// Token rows per stage (a chunk), by conv width.
+template <int W>
+__host__ __device__ constexpr int prefill_rows() {
+  return W <= 4 ? SCONV_PREFILL_ROWS_SMALL_W : SCONV_PREFILL_ROWS;
+}
+inline int prefill_rows(int W) { return W <= 4 ? SCONV_PREFILL_ROWS_SMALL_W : SCONV_PREFILL_ROWS; }
 
 // Measured on B200: with W <= 4 (two CTAs per SM, 128 registers) the fast
 // path is unrolled by 4 and gamma is read from shared memory per token,
@@ -115,7 +123,9 @@ constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 4;
 // bytes (the row layout keeps that fixed pitch between rows, so a thread's
 // per-token shared-memory loads take immediate offsets).
 constexpr int kTmaRowPitch = kTmaMaxGroups * 16;
-constexpr int kTmaStageBytes = kTmaRows * kTmaRowPitch;
+template <int W>
+__host__ __device__ constexpr int prefill_stage_bytes() { return prefill_rows<W>() * kTmaRowPitch; }
+inline int prefill_stage_bytes(int W) { return prefill_rows(W) * kTmaRowPitch; }
 constexpr int kTmaGammaBytes = kTmaMaxGroups * 32;  // 8 gammas per thread (W <= 4)
 
 struct TmaGeom {
@@ -207,7 +217,8 @@ __device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 
 template <int W, int D, bool MX, bool LV>
 __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom& Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int R = kTmaRows;
+  constexpr int R = prefill_rows<W>();
+  constexpr int kTmaStageBytes = prefill_stage_bytes<W>();
   // layout variants (per-head gamma stride, ring-buffer state) only in the
   // LV instances: elsewhere these fold to the defaults at compile time, so
   // the default path carries no extra live values

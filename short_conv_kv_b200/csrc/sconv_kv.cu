@@ -307,7 +307,7 @@ int prefill_impl(
   sconv::TmaGeom G;
   G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
-  const int stage_bytes = sconv::kTmaStageBytes;  // laid out for a full slice
+  const int stage_bytes = sconv::prefill_stage_bytes(W);  // laid out for a full slice
   const int per_sm = sconv::prefill_ctas_per_sm(W, mx);
   int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
@@ -339,7 +339,8 @@ int prefill_impl(
                                   smem, per_sm);
   const int64_t resident = static_cast<int64_t>(sm_count()) * (occ < per_sm ? occ : per_sm);
   int64_t ctas = resident / ctas_y;
-  const int64_t by_tokens = (num_tokens + sconv::kTmaRows - 1) / sconv::kTmaRows;
+  const int R = sconv::prefill_rows(W);
+  const int64_t by_tokens = (num_tokens + R - 1) / R;
   if (ctas > by_tokens) ctas = by_tokens;
   if (ctas < 1) ctas = 1;
   G.ctas = static_cast<int>(ctas);
