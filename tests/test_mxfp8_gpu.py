@@ -152,3 +152,78 @@ def test_mx_rejects_unaligned_layout():
                                 gu.dev(b.conv_w_k), gu.dev(b.conv_w_v), gu.dev(b.gamma_k),
                                 gu.dev(b.gamma_v), b.eps, gu.dev(b.conv_state),
                                 gu.dev(b.slot_mapping), kd, ks[:, :, :, :1], kd.clone(), ks)
+
+
+def test_mx_chunks_back_to_back_state_only_dependency():
+    """Five chunks of one sequence (3,000 tokens each) through the MXFP8
+    store, launched back to back with the state-only dependency and no
+    synchronisation in between; each chunk against the oracle run on the
+    state the previous chunk left, and the final state bit for bit."""
+    b = _binding()
+    n, L = 5, 3000
+    chunks = [wl.make_prefill([L], Hkv=8, D=128, W=4, seed=1900 + c, state="zero", page_size=16,
+                              spare_pages=0) for c in range(n)]
+    base = chunks[0]
+    for x in chunks:
+        x.conv_w_k, x.conv_w_v, x.gamma_k, x.gamma_v = (base.conv_w_k, base.conv_w_v,
+                                                        base.gamma_k, base.gamma_v)
+    st = gu.dev(base.conv_state.clone())
+    w = [gu.dev(t) for t in (base.conv_w_k, base.conv_w_v, base.gamma_k, base.gamma_v)]
+    caches = [gu.mx_caches(x.num_pages, x.page_size, x.Hkv, x.D) + gu.mx_caches(
+        x.num_pages, x.page_size, x.Hkv, x.D) for x in chunks]
+    devs = [(gu.dev(x.k), gu.dev(x.v), gu.dev(x.cu_seqlens), gu.dev(x.slot_mapping)) for x in chunks]
+    torch.cuda.synchronize()
+    for (k, v, cu, sm), (kd, ks, vd, vs) in zip(devs, caches):
+        b.prefill_varlen_mxfp8(k, v, cu, *w, base.eps, st, sm, kd, ks, vd, vs,
+                               state_only_dependency=True)
+    torch.cuda.synchronize()
+    state = wl.bits(base.conv_state)
+    for c, (x, (kd, ks, vd, vs)) in enumerate(zip(chunks, caches)):
+        x.conv_state = wl.from_bits(state)
+        ref = gu.oracle_prefill(x)
+        sm = x.slot_mapping.numpy()
+        gu.check_mx(kd.cpu().numpy(), ks.cpu().numpy(), sm, ref["z_k"], f"k mx chunk {c}")
+        gu.check_mx(vd.cpu().numpy(), vs.cpu().numpy(), sm, ref["z_v"], f"v mx chunk {c}")
+        state = ref["conv_state"]
+    assert np.array_equal(wl.bits(st.cpu()), state)
+
+
+def test_mx_decode_independent_state_alternating():
+    """MXFP8 decode: two batches on disjoint state rows of one pool,
+    launched alternately with the independent-state promise, 6 steps each,
+    no synchronisation in between; every step against the oracle chain."""
+    b = _binding()
+    B, steps = 128, 6
+    setups = [wl.decode(seed=7300 + j, batch=B, pages_per_seq=1, page_size=16, max_start=8)
+              for j in range(2)]
+    sA = setups[0]
+    pool = torch.cat([s.conv_state for s in setups])
+    st = gu.dev(pool.clone())
+    idx = [gu.dev(torch.arange(j * B, (j + 1) * B, dtype=torch.int32)) for j in range(2)]
+    w = [gu.dev(x) for x in (sA.conv_w_k, sA.conv_w_v, sA.gamma_k, sA.gamma_v)]
+    caches = [[gu.mx_caches(s.num_pages, s.page_size, s.Hkv, s.D) + gu.mx_caches(
+        s.num_pages, s.page_size, s.Hkv, s.D) for _ in range(steps)] for s in setups]
+    inputs = [[s.step_inputs(t) for t in range(steps)] for s in setups]
+    dev_in = [[tuple(gu.dev(x) for x in inp) for inp in seq] for seq in inputs]
+    torch.cuda.synchronize()
+    for t in range(steps):
+        for j in range(2):
+            k, v, sm = dev_in[j][t]
+            b.decode_mxfp8(k, v, *w, sA.eps, st, sm, *caches[j][t], state_indices=idx[j],
+                           independent_state=True)
+    torch.cuda.synchronize()
+    small = np.zeros((B, 1, sA.Hkv, sA.D), np.uint16)
+    for j, s in enumerate(setups):
+        ref_state = wl.bits(s.conv_state)
+        for t in range(steps):
+            k, v, sm = inputs[j][t]
+            ref = oracle.decode(wl.bits(k), wl.bits(v), wl.bits(sA.conv_w_k), wl.bits(sA.conv_w_v),
+                                sA.gamma_k.numpy(), sA.gamma_v.numpy(), sA.eps, ref_state,
+                                np.arange(B, dtype=np.int64), small, small.copy())
+            ref_state = ref["conv_state"]
+            kd, ks, vd, vs = caches[j][t]
+            smn = sm.numpy()
+            gu.check_mx(kd.cpu().numpy(), ks.cpu().numpy(), smn, ref["z_k"], f"k {j} {t}")
+            gu.check_mx(vd.cpu().numpy(), vs.cpu().numpy(), smn, ref["z_v"], f"v {j} {t}")
+        got = wl.bits(st.cpu())[j * B:(j + 1) * B]
+        assert np.array_equal(got, ref_state), f"state of batch {j}"
