@@ -52,19 +52,29 @@ namespace sconv {
 #ifndef SCONV_PREFILL_SMALL_W_PER_SM
 #define SCONV_PREFILL_SMALL_W_PER_SM 2  // CTAs per SM for W <= 4
 #endif
+#ifndef SCONV_PREFILL_BF16_THREADS
+#define SCONV_PREFILL_BF16_THREADS 256  // threads per CTA of the bf16 store for W <= 4
+#endif
 #ifndef SCONV_PREFILL_BF16_UNROLL
 #define SCONV_PREFILL_BF16_UNROLL 4  // fast-path unroll of the bf16 store for W <= 4
 #endif
 #ifndef SCONV_PREFILL_MX_UNROLL
 #define SCONV_PREFILL_MX_UNROLL 8  // fast-path unroll of the MXFP8 store for W <= 4
 #endif
+// The MXFP8 store for W <= 4: threads per CTA (= channel groups per slice)
+// and CTAs per SM.  Measured on B200, with an 8-token unroll and gammas in
+// registers: three 128-thread CTAs per SM (166 registers, 12 warps)
+// against one 256-thread CTA (211 registers, 8 warps): 65,536-token launch
+// 92.2 -> 85.3 us, varlen batch 198.2 -> 184.6 us, 8192-token launch
+// 18.0 -> 17.7 us; one 256-thread CTA in turn beat two with a 2-token
+// unroll (102.1 -> 92.2 us).  The MX store's per-token chain is longer
+// than the bf16 store's: the launch is issue-latency-bound, and both the
+// wider unroll and the extra warps hide it.
+#ifndef SCONV_PREFILL_MX_THREADS
+#define SCONV_PREFILL_MX_THREADS 128
+#endif
 #ifndef SCONV_PREFILL_MX_PER_SM
-// CTAs per SM of the MXFP8 store for W <= 4.  Measured on B200: one CTA
-// per SM with an 8-token unroll and gammas in registers (211 registers)
-// against two with a 2-token unroll: 65,536-token launch 102.1 -> 91.9 us,
-// 8192-token launch 19.1 -> 18.0 us, varlen batch 220.5 -> 197.4 us (the
-// MX store's longer per-token chain needs the wider unroll).
-#define SCONV_PREFILL_MX_PER_SM 1
+#define SCONV_PREFILL_MX_PER_SM 3
 #endif
 #ifndef SCONV_PREFILL_FIRST_FILL
 // Chunks requested before the first one has landed (0 = the whole ring);
@@ -97,8 +107,20 @@ template <int W, bool MX>
 __host__ __device__ constexpr int prefill_ctas_per_sm() {
   return W <= 4 ? (MX ? SCONV_PREFILL_MX_PER_SM : SCONV_PREFILL_SMALL_W_PER_SM) : 1;
 }
+// Threads per CTA, one per channel group of the CTA's slice.
 template <int W, bool MX>
-__host__ __device__ constexpr bool gamma_in_smem() { return prefill_ctas_per_sm<W, MX>() > 1; }
+__host__ __device__ constexpr int prefill_threads() {
+  return W <= 4 ? (MX ? SCONV_PREFILL_MX_THREADS : SCONV_PREFILL_BF16_THREADS) : kTmaMaxGroups;
+}
+inline int prefill_threads(int W, bool mx) {
+  return W <= 4 ? (mx ? SCONV_PREFILL_MX_THREADS : SCONV_PREFILL_BF16_THREADS) : kTmaMaxGroups;
+}
+// gammas read from shared memory per token: when an SM holds 512 threads
+// or more (at most 128 registers each) there is no room to hold them
+template <int W, bool MX>
+__host__ __device__ constexpr bool gamma_in_smem() {
+  return prefill_threads<W, MX>() * prefill_ctas_per_sm<W, MX>() >= 512;
+}
 template <int W, bool MX>
 __host__ __device__ constexpr int fast_unroll() {
   return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : SCONV_PREFILL_BF16_UNROLL) : 8;
@@ -119,17 +141,28 @@ constexpr int kTmaCuSmemMax = 2048;  // cu_seqlens entries staged in shared memo
 // refuses caches whose row offsets do not fit
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 constexpr int kTmaOffTableBytes = (kTmaMaxGroups / 32) * 32 * 4;
-// Every stage is laid out for a full slice: R rows of kTmaMaxGroups * 16
-// bytes (the row layout keeps that fixed pitch between rows, so a thread's
-// per-token shared-memory loads take immediate offsets).
-constexpr int kTmaRowPitch = kTmaMaxGroups * 16;
-template <int W>
-__host__ __device__ constexpr int prefill_stage_bytes() { return prefill_rows<W>() * kTmaRowPitch; }
-inline int prefill_stage_bytes(int W) { return prefill_rows(W) * kTmaRowPitch; }
-constexpr int kTmaGammaBytes = kTmaMaxGroups * 32;  // 8 gammas per thread (W <= 4)
+// Every stage is laid out for a full slice: R rows of (threads per CTA) *
+// 16 bytes (the row layout keeps that fixed pitch between rows, so a
+// thread's per-token shared-memory loads take immediate offsets).
+template <int W, bool MX>
+__host__ __device__ constexpr int prefill_row_pitch() { return prefill_threads<W, MX>() * 16; }
+template <int W, bool MX>
+__host__ __device__ constexpr int prefill_stage_bytes() {
+  return prefill_rows<W>() * prefill_row_pitch<W, MX>();
+}
+inline int prefill_stage_bytes(int W, bool mx) { return prefill_rows(W) * prefill_threads(W, mx) * 16; }
+// per-thread gammas in shared memory (8 floats per thread), when used
+template <int W, bool MX>
+__host__ __device__ constexpr int prefill_gamma_bytes() {
+  return gamma_in_smem<W, MX>() ? prefill_threads<W, MX>() * 32 : 0;
+}
+inline int prefill_gamma_bytes(int W, bool mx) {
+  const int per_sm = W <= 4 ? (mx ? SCONV_PREFILL_MX_PER_SM : SCONV_PREFILL_SMALL_W_PER_SM) : 1;
+  return prefill_threads(W, mx) * per_sm >= 512 ? prefill_threads(W, mx) * 32 : 0;
+}
 
 struct TmaGeom {
-  int slice;      // channel groups per full slice (min(NG, 256))
+  int slice;      // channel groups per full slice (min(NG, threads per CTA))
   int stages;     // ring depth
   int ctas;       // persistent CTAs along the token axis
   int withhold_first;  // testing: chunk 0 is never requested (its wait runs out)
@@ -218,7 +251,9 @@ template <int W, int D, bool MX, bool LV>
 __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom& Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int R = prefill_rows<W>();
-  constexpr int kTmaStageBytes = prefill_stage_bytes<W>();
+  constexpr int kTmaStageBytes = prefill_stage_bytes<W, MX>();
+  constexpr int kTmaRowPitch = prefill_row_pitch<W, MX>();
+  constexpr int kTmaGammaBytes = prefill_gamma_bytes<W, MX>();
   // layout variants (per-head gamma stride, ring-buffer state) only in the
   // LV instances: elsewhere these fold to the defaults at compile time, so
   // the default path carries no extra live values
@@ -716,7 +751,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
 }
 
 template <int W, int D, int MINB, bool MX, bool LV>
-__global__ void __launch_bounds__(kTmaMaxGroups, MINB)
+__global__ void __launch_bounds__(prefill_threads<W, MX>(), MINB)
     prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
   prefill_body<W, D, MX, LV>(P, Gm);
   // With the state-only dependency a CTA that never touched a state row has

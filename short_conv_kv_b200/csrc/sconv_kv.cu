@@ -305,14 +305,17 @@ int prefill_impl(
   // are resident (x), each streaming a contiguous token range of at least
   // one stage.
   sconv::TmaGeom G;
-  G.slice = P.NG < sconv::kTmaMaxGroups ? P.NG : sconv::kTmaMaxGroups;
+  const int nt = sconv::prefill_threads(W, mx);  // threads (channel groups) per CTA
+  G.slice = P.NG < nt ? P.NG : nt;
   const int ctas_y = (P.NG + G.slice - 1) / G.slice;
-  const int stage_bytes = sconv::prefill_stage_bytes(W);  // laid out for a full slice
+  const int stage_bytes = sconv::prefill_stage_bytes(W, mx);  // laid out for a full slice
   const int per_sm = sconv::prefill_ctas_per_sm(W, mx);
-  int stages = (per_sm == 2 ? sconv::kTmaRingBytes2 : 2 * sconv::kTmaRingBytes2) / stage_bytes;
+  // the ring: 192 KB of an SM's shared memory split among its CTAs
+  int stages = (2 * sconv::kTmaRingBytes2 / per_sm) / stage_bytes;
   G.stages = stages < 2 ? 2 : (stages > 16 ? 16 : stages);
   // + per-warp slot-offset tables + per-thread gammas
-  G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes + sconv::kTmaGammaBytes;
+  G.smem_ring = G.stages * stage_bytes + sconv::kTmaOffTableBytes +
+                sconv::prefill_gamma_bytes(W, mx);
   // cu_seqlens is staged in shared memory only while per_sm CTAs still fit
   // on an SM with it (beyond that the CTAs read it from global memory):
   // staging must never cost a resident CTA
