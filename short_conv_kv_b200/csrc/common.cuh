@@ -159,14 +159,14 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 
 // Quantise this lane's 8 normalised values z = t * r (t = conv output times
 // gamma, r = the head's 1/rms; channels d0..d0+7 of a head) as part of their
-// 32-channel block and store: 8 code bytes at `data`, and (lane % 4 == 0
-// of the block's 4 lanes) the E8M0 scale byte at `scale`.  z is formed
+// 32-channel block: the 8 E4M3 codes (w0: channels 0-3, w1: 4-7, low
+// element in the low byte) and the block's E8M0 scale byte sb.  z is formed
 // first and then scaled by the exact power of two 2^-s (<= 2^127, and
 // |z| * 2^-s < 512, so nothing overflows; folding 2^-s into r instead would
 // overflow for all-zero blocks).  All 32 lanes of the warp must call it
-// (shuffles); `write` masks the stores.
-__device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool write,
-                                          uint8_t* data, uint8_t* scale) {
+// (shuffles over each block's 4 lanes).
+__device__ __forceinline__ void mx_encode8(const float2 (&t)[4], float r, uint32_t& w0,
+                                           uint32_t& w1, uint32_t& sb) {
   const float2 rr = make_float2(r, r);
   const float2 z[4] = {__fmul2_rn(t[0], rr), __fmul2_rn(t[1], rr), __fmul2_rn(t[2], rr),
                        __fmul2_rn(t[3], rr)};
@@ -175,13 +175,21 @@ __device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool wr
   float amax = fmaxf(m1, max_abs3(z[3].x, z[3].y, m0));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-  const uint32_t sb = mx_scale_byte(amax);
+  sb = mx_scale_byte(amax);
   const float m = mx_inv_scale(sb);  // 2^-s, exact
   const float2 mm = make_float2(m, m);
   const float2 a = __fmul2_rn(z[0], mm), b = __fmul2_rn(z[1], mm);
   const float2 c = __fmul2_rn(z[2], mm), d = __fmul2_rn(z[3], mm);
-  const uint32_t w0 = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
-  const uint32_t w1 = e4m3x2(c.x, c.y) | (e4m3x2(d.x, d.y) << 16);
+  w0 = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+  w1 = e4m3x2(c.x, c.y) | (e4m3x2(d.x, d.y) << 16);
+}
+
+// mx_encode8, then the store: 8 code bytes at `data`, and (lane % 4 == 0
+// of the block's 4 lanes) the scale byte at `scale`; `write` masks both.
+__device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool write,
+                                          uint8_t* data, uint8_t* scale) {
+  uint32_t w0, w1, sb;
+  mx_encode8(t, r, w0, w1, sb);
   const bool scale_writer = write && ((threadIdx.x & 3) == 0);
   asm volatile(
       "{\n\t.reg .pred q, r;\n\t"
@@ -190,6 +198,35 @@ __device__ __forceinline__ void mx_store8(const float2 (&t)[4], float r, bool wr
       "@q st.global.cs.v2.u32 [%2], {%3, %4};\n\t"
       "@r st.global.cs.u8 [%5], %6;\n\t}" ::"r"(static_cast<int>(write)),
       "r"(static_cast<int>(scale_writer)), "l"(data), "r"(w0), "r"(w1), "l"(scale), "r"(sb)
+      : "memory");
+}
+
+// Row stores addressed by a cache row offset in units of 8 elements
+// (`off8`; 0xFFFFFFFF: the row is not written, and the store is skipped).
+// bf16: the 16 bytes at base + off8 * 16.
+__device__ __forceinline__ void st_row_bf16(uint32_t off8, uint16_t* base, const uint4& v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t.reg .u64 a;\n\t"
+      "setp.ne.u32 q, %0, -1;\n\t"
+      "mad.wide.u32 a, %0, 16, %1;\n\t"
+      "@q st.global.cs.v4.u32 [a], {%2, %3, %4, %5};\n\t}" ::"r"(off8),
+      "l"(base), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+      : "memory");
+}
+// MXFP8: the 8 code bytes at data + off8 * 8 and, where scale_lane is
+// nonzero, the scale byte at scale + off8 / 4.
+__device__ __forceinline__ void st_row_mx(uint32_t off8, uint8_t* data, uint8_t* scale,
+                                          int scale_lane, uint32_t w0, uint32_t w1, uint32_t sb) {
+  asm volatile(
+      "{\n\t.reg .pred q, r;\n\t.reg .u32 o;\n\t.reg .u64 a, b;\n\t"
+      "setp.ne.u32 q, %0, -1;\n\t"
+      "setp.ne.and.b32 r, %1, 0, q;\n\t"
+      "mad.wide.u32 a, %0, 8, %2;\n\t"
+      "shr.u32 o, %0, 2;\n\t"
+      "mad.wide.u32 b, o, 1, %3;\n\t"
+      "@q st.global.cs.v2.u32 [a], {%4, %5};\n\t"
+      "@r st.global.cs.u8 [b], %6;\n\t}" ::"r"(off8),
+      "r"(scale_lane), "l"(data), "l"(scale), "r"(w0), "r"(w1), "r"(sb)
       : "memory");
 }
 

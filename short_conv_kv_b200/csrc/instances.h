@@ -25,6 +25,9 @@ inline int prefill_ctas_per_sm(int W, bool mx) {
 TmaFn pick_prefill_bf16(int W, int D);
 TmaFn pick_prefill_mx(int W, int D);
 TmaFn pick_prefill_bf16_lv(int W, int D);
+// bf16 store, W <= 4, for short launches (SCONV_PREFILL_SHORT_CHUNKS in
+// prefill_tma.cuh); nullptr for W > 4
+TmaFn pick_prefill_bf16_short(int W, int D);
 TmaFn pick_prefill_mx_lv(int W, int D);
 DecFn pick_decode(int W, int D, bool mx, bool lv);
 

@@ -58,6 +58,30 @@ namespace sconv {
 #ifndef SCONV_PREFILL_BF16_UNROLL
 #define SCONV_PREFILL_BF16_UNROLL 4  // fast-path unroll of the bf16 store for W <= 4
 #endif
+// Fast-path tokens per batched head reduction (head_rsqrt_batch).  Measured
+// on B200 against batches of 4 (bf16, W <= 4 and MXFP8) and 8 (W > 4), one
+// box, back to back: 65,536 tokens at W=8 101.1 -> 98.6 us, MXFP8 chunk
+// 80.7 -> 80.1 us, MXFP8 varlen 178.4 -> 176.4 us, bf16 chunk 93.1 ->
+// 92.3 us, bf16 varlen 206.5 -> 203.8 us (the shorter dependent shuffle
+// chain hides better); the bf16 8192-token launch is the opposite case
+// (15.6 against 16.1 us) and has its own instance (SCONV_PREFILL_SHORT_*).
+#ifndef SCONV_PREFILL_NORM_BATCH
+#define SCONV_PREFILL_NORM_BATCH 2
+#endif
+#ifndef SCONV_PREFILL_MX_NORM_BATCH
+#define SCONV_PREFILL_MX_NORM_BATCH 2  // the same for the MXFP8 store, W <= 4
+#endif
+// Short launches (at most SCONV_PREFILL_SHORT_CHUNKS chunks per CTA) of the
+// bf16 W <= 4 store: every CTA's chunks land at about the same time and the
+// launch ends in a compute-bound tail, where fewer instructions per token
+// count more than the reduction's latency: that instance reduces 4 tokens
+// at a time.
+#ifndef SCONV_PREFILL_SHORT_CHUNKS
+#define SCONV_PREFILL_SHORT_CHUNKS 8
+#endif
+#ifndef SCONV_PREFILL_SHORT_NORM_BATCH
+#define SCONV_PREFILL_SHORT_NORM_BATCH 4
+#endif
 #ifndef SCONV_PREFILL_MX_UNROLL
 #define SCONV_PREFILL_MX_UNROLL 8  // fast-path unroll of the MXFP8 store for W <= 4
 #endif
@@ -121,9 +145,24 @@ template <int W, bool MX>
 __host__ __device__ constexpr bool gamma_in_smem() {
   return prefill_threads<W, MX>() * prefill_ctas_per_sm<W, MX>() >= 512;
 }
-template <int W, bool MX>
+// (the W=3 and W=4 bf16 layout-variant instances carry two more live
+// values at their 128-register cap: there only a 2-token unroll and batch
+// stay free of spills for every head size)
+template <int W, bool MX, bool LV = false>
 __host__ __device__ constexpr int fast_unroll() {
-  return W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : SCONV_PREFILL_BF16_UNROLL) : 8;
+  return (W >= 3 && W <= 4 && !MX && LV) ? 2
+         : W <= 4 ? (MX ? SCONV_PREFILL_MX_UNROLL : SCONV_PREFILL_BF16_UNROLL) : 8;
+}
+// tokens whose head reductions run together in the fast path (a divisor
+// of the unroll)
+// NBX > 0: an instance's own batch (the short-launch instances)
+template <int W, bool MX, bool LV, int NBX = 0>
+__host__ __device__ constexpr int norm_batch() {
+  return NBX > 0 ? NBX
+         : (W <= 4 && MX) ? SCONV_PREFILL_MX_NORM_BATCH
+         : (W >= 3 && W <= 4 && !MX && LV) ? 2
+         : SCONV_PREFILL_NORM_BATCH < fast_unroll<W, MX>() ? SCONV_PREFILL_NORM_BATCH
+                                                           : fast_unroll<W, MX>();
 }
 // Measured on B200: the block layout (2 bulk copies per chunk instead of
 // 2 per row) speeds up the wide-window and MXFP8 instances by 14-25 %; in
@@ -175,10 +214,18 @@ struct TmaGeom {
   unsigned long long timeout_ns;
 };
 
-// Per-token work of one thread: conv of its 8 channels over the window and
-// the new row, then the window shift.  Returns the conv output in acc.
+// Per-token work of one thread: the conv of its 8 channels, in transposed
+// form.  part[k-1] holds P_k, the part of the output k tokens ahead that the
+// rows seen so far contribute: P_k = w_0 x_{t+k-W+1} + ... + w_{W-1-k} x_t,
+// summed in tap order.  A new row x_t completes y_t = w_{W-1} x_t + P_1 and
+// extends every other partial by one tap, P_k <- w_{W-1-k} x_t + P_{k+1}
+// (P_{W-1} <- w_0 x_t).  Each output is thus the same chain of fused
+// multiply-adds, in the same tap order, as the direct sum over the window
+// w_0 x_{t-W+1} + ... + w_{W-1} x_t, and bitwise equal to it; the carried
+// values are produced in place, so no window rows are shifted between
+// tokens.  Returns the conv output in acc.
 template <int W>
-__device__ __forceinline__ void conv_step(const float2 (&tw)[W][4], float2 (&win)[W > 1 ? W - 1 : 1][4],
+__device__ __forceinline__ void conv_step(const float2 (&tw)[W][4], float2 (&part)[W > 1 ? W - 1 : 1][4],
                                           const uint4& xr, float2 (&acc)[4]) {
   float2 xf[4];
   unpack8(xr, xf);
@@ -187,19 +234,101 @@ __device__ __forceinline__ void conv_step(const float2 (&tw)[W][4], float2 (&win
     if constexpr (W == 1) {
       acc[e] = fmul2(tw[0][e], xf[e]);
     } else {
-      acc[e] = fmul2(tw[0][e], win[0][e]);
+      acc[e] = ffma2(tw[W - 1][e], xf[e], part[0][e]);
 #pragma unroll
-      for (int j = 1; j < W - 1; ++j) acc[e] = ffma2(tw[j][e], win[j][e], acc[e]);
-      acc[e] = ffma2(tw[W - 1][e], xf[e], acc[e]);
+      for (int k = 1; k < W - 1; ++k) part[k - 1][e] = ffma2(tw[W - 1 - k][e], xf[e], part[k][e]);
+      part[W - 2][e] = fmul2(tw[0][e], xf[e]);
     }
   }
+}
+
+// The partials P_1 .. P_{W-1} of the window's W-1 rows in front of a token
+// (h[0] oldest), built tap by tap in the order conv_step extends them.
+template <int W>
+__device__ __forceinline__ void conv_prime(const float2 (&tw)[W][4], const uint4 (&hb)[W > 1 ? W - 1 : 1],
+                                           float2 (&part)[W > 1 ? W - 1 : 1][4]) {
   if constexpr (W > 1) {
+    float2 h[W - 1][4];
 #pragma unroll
-    for (int j = 0; j < W - 2; ++j)
+    for (int j = 0; j < W - 1; ++j) unpack8(hb[j], h[j]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) win[j][e] = win[j + 1][e];
+    for (int k = 1; k < W; ++k)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) win[W - 2][e] = xf[e];
+      for (int e = 0; e < 4; ++e) {
+        float2 p = fmul2(tw[0][e], h[k - 1][e]);
+#pragma unroll
+        for (int j = 1; j < W - k; ++j) p = ffma2(tw[j][e], h[k + j - 1][e], p);
+        part[k - 1][e] = p;
+      }
+  }
+}
+
+// Sum of squares of this lane's 8 conv outputs (even and odd lanes of the
+// packed pairs summed separately, then added).
+__device__ __forceinline__ float sum_sq8(const float2 (&acc)[4]) {
+  float2 s2 = fmul2(acc[0], acc[0]);
+  s2 = ffma2(acc[1], acc[1], s2);
+  s2 = ffma2(acc[2], acc[2], s2);
+  s2 = ffma2(acc[3], acc[3], s2);
+  return s2.x + s2.y;
+}
+
+// 1/rms of NB tokens at once: v[t] holds this lane's sum of squares of
+// token t; r[t] receives rsqrt(total over the lane's group of G lanes *
+// inv_d + eps) on every lane.  The first log2(min(NB, G)) butterfly levels
+// halve the values a lane carries: of each pair of tokens it keeps the one
+// its lane bit at that level selects and adds the partner lane's partial of
+// that token; the remaining levels are plain.  Every addition joins the same
+// two lane sets as group_sum's butterfly (own partial + partner's), so each
+// total is bitwise the one group_sum gives.  One rsqrt per lane, then each
+// token's value is fetched from a lane that holds it (shfl.idx whose
+// segment mask keeps the lane's own bits outside the selecting ones).
+template <int G, int NB>
+__device__ __forceinline__ void head_rsqrt_batch(float (&v)[NB], float inv_d, float eps, float (&r)[NB]) {
+  constexpr int LG = G >= 32 ? 5 : G >= 16 ? 4 : G >= 8 ? 3 : G >= 4 ? 2 : G >= 2 ? 1 : 0;
+  constexpr int LN = NB >= 8 ? 3 : NB >= 4 ? 2 : NB >= 2 ? 1 : 0;
+  static_assert((1 << LG) == G && (1 << LN) == NB, "powers of two");
+  constexpr int H = LN < LG ? LN : LG;  // halving levels
+  constexpr int NL = NB >> H;           // values left per lane
+#pragma unroll
+  for (int i = 0; i < H; ++i) {
+    const int m = G >> (i + 1);
+    const bool hi = (threadIdx.x & m) != 0;
+    const int half = NB >> (i + 1);
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float a = v[k], b = v[k + half];
+      const float keep = hi ? b : a;
+      const float send = hi ? a : b;
+      v[k] = keep + __shfl_xor_sync(kFullMask, send, m);
+    }
+  }
+  float own[NL];
+#pragma unroll
+  for (int k = 0; k < NL; ++k) {
+    float x = v[k];
+#pragma unroll
+    for (int m = G >> (H + 1); m >= 1; m >>= 1) x += __shfl_xor_sync(kFullMask, x, m);
+    own[k] = rsqrt_approx(fmaf(x, inv_d, eps));
+  }
+  // token t = k + sum_i b_i * (NB >> (i+1)), b_i the lane bit at position
+  // LG-1-i: its holders have those bits, any others
+  constexpr int kSel = ((1 << LG) - 1) & ~((1 << (LG - H)) - 1);
+  constexpr unsigned kC = ((0x1fu & ~static_cast<unsigned>(kSel)) << 8) | 0x1fu;
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    int bits = 0;
+#pragma unroll
+    for (int i = 0; i < H; ++i)
+      if ((t / (NB >> (i + 1))) & 1) bits |= 1 << (LG - 1 - i);
+    if constexpr (H == 0) {
+      r[t] = own[t];
+    } else {
+      float y;
+      asm volatile("shfl.sync.idx.b32 %0, %1, %2, %3, 0xffffffff;"
+                   : "=f"(y) : "f"(own[t % NL]), "r"(bits), "n"(kC));
+      r[t] = y;
+    }
   }
 }
 
@@ -219,35 +348,51 @@ __device__ __forceinline__ void lds_gamma(const float* g, float2 (&gm)[4]) {
   gm[3] = make_float2(b.z, b.w);
 }
 
-// RMSNorm of the head (D/8 lanes), gamma, then either bf16 rounding and a
+// NB consecutive entries of a slot table (16-byte aligned for NB >= 4,
+// NB * 4 bytes aligned below that) in as few shared-memory loads as fit.
+template <int NB>
+__device__ __forceinline__ void load_offsets(const uint32_t* p, uint32_t (&o)[NB]) {
+  if constexpr (NB % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NB; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+      o[i] = v.x; o[i + 1] = v.y; o[i + 2] = v.z; o[i + 3] = v.w;
+    }
+  } else if constexpr (NB == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    o[0] = v.x; o[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < NB; ++i) o[i] = p[i];
+  }
+}
+
+// Gamma and the head's 1/rms applied, then either bf16 rounding and a
 // 16-byte store into the bf16 cache (MX = false), or the MXFP8 block store
-// (8 E4M3 bytes + the block's E8M0 scale).
-template <int D, bool MX>
-__device__ __forceinline__ void norm_store(const float2 (&acc)[4], const float2 (&gm)[4],
-                                           float inv_d, float eps, bool write,
-                                           uint16_t* dst, uint8_t* mx_data, uint8_t* mx_scale) {
-  float2 s2 = fmul2(acc[0], acc[0]);
-  s2 = ffma2(acc[1], acc[1], s2);
-  s2 = ffma2(acc[2], acc[2], s2);
-  s2 = ffma2(acc[3], acc[3], s2);
-  const float ss = group_sum<D / 8>(s2.x + s2.y);
-  const float rn = rsqrt_approx(fmaf(ss, inv_d, eps));
+// (8 E4M3 bytes + the block's E8M0 scale), at cache row offset off8 (units
+// of 8 elements; kNoRow: not written).
+template <bool MX>
+__device__ __forceinline__ void scale_store(const float2 (&acc)[4], const float2 (&gm)[4], float rn,
+                                            uint32_t off8, uint16_t* cache, uint8_t* mx_data,
+                                            uint8_t* mx_scale, int scale_lane) {
   const float2 rr = make_float2(rn, rn);
   if constexpr (MX) {
     const float2 t[4] = {fmul2(acc[0], gm[0]), fmul2(acc[1], gm[1]), fmul2(acc[2], gm[2]),
                          fmul2(acc[3], gm[3])};
-    mx_store8(t, rn, write, mx_data, mx_scale);
+    uint32_t w0, w1, sb;
+    mx_encode8(t, rn, w0, w1, sb);
+    st_row_mx(off8, mx_data, mx_scale, scale_lane, w0, w1, sb);
   } else {
     uint4 o;
     o.x = pack_bf16x2(fmul2(fmul2(acc[0], rr), gm[0]));
     o.y = pack_bf16x2(fmul2(fmul2(acc[1], rr), gm[1]));
     o.z = pack_bf16x2(fmul2(fmul2(acc[2], rr), gm[2]));
     o.w = pack_bf16x2(fmul2(fmul2(acc[3], rr), gm[3]));
-    st_stream_if(write, dst, o);
+    st_row_bf16(off8, cache, o);
   }
 }
 
-template <int W, int D, bool MX, bool LV>
+template <int W, int D, bool MX, bool LV, int NBX>
 __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom& Gm) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int R = prefill_rows<W>();
@@ -510,12 +655,13 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
       gm[3] = make_float2(b.z, b.w);
     }
   }
+  // the conv's carried partials (conv_step), set at each sequence start
   constexpr int NH = W > 1 ? W - 1 : 1;
-  float2 win[NH][4];
+  float2 part[NH][4];
 #pragma unroll
   for (int j = 0; j < NH; ++j)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) win[j][e] = make_float2(0.f, 0.f);
+    for (int e = 0; e < 4; ++e) part[j][e] = make_float2(0.f, 0.f);
 
   int seq = seq0;
   int next = (seq + 1 <= S) ? cu(seq + 1) : T;
@@ -591,8 +737,7 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < W - 1; ++j) unpack8(hb[j], win[j]);
+      conv_prime<W>(tw, hb, part);
     }
   };
 
@@ -605,29 +750,55 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
       // halo: rows first_row-(W-1) .. first_row-1.  When first_row == ta
       // (the cut did not move) they lie in ta's sequence at positions >= 0,
       // never in the state; otherwise they only feed the masked rows.
+      uint4 hb[W - 1];
 #pragma unroll
       for (int j = 0; j < W - 1; ++j) {
         const int64_t q = static_cast<int64_t>(first_row) - (W - 1) + j;
-        const uint4 h = (active && q >= 0) ? ld_ro(xbase + q * P.row_stride) : make_uint4(0, 0, 0, 0);
-        unpack8(h, win[j]);
+        hb[j] = (active && q >= 0) ? ld_ro(xbase + q * P.row_stride) : make_uint4(0, 0, 0, 0);
       }
+      conv_prime<W>(tw, hb, part);
     }
   }
 
   const float eps = P.eps, inv_d = P.inv_d;
-  // `off8`: the row's cache offset in units of 8 elements (bf16: 16 bytes;
-  // MXFP8: 8 code bytes, and a quarter of a scale byte), kNoRow if unwritten
-#define NORM_STORE(pred)                                                            \
+  // A row's cache offset is kept in units of 8 elements (bf16: 16 bytes;
+  // MXFP8: 8 code bytes, and a quarter of a scale byte), kNoRow if the row
+  // is not written; lanes outside the slice force every offset to kNoRow.
+  // (vector loads of a batch's offsets only where registers are plentiful:
+  // at the 128-register cap of the bf16 W <= 4 instances they spill)
+  constexpr bool kVecOffsets = !gamma_in_smem<W, MX>();
+  const int scale_lane = (threadIdx.x & 3) == 0;  // MXFP8: writes its block's scale
+#define SCALE_STORE(a, rn, gs, off)                                                 \
+  scale_store<MX>(a, gs, rn, off, cache, mxdata, mxscale, scale_lane)
+  // one token (sequence starts, partial chunks): its head's 1/rms, the store
+#define NORM_STORE(off)                                                             \
   do {                                                                              \
-    uint8_t* mxd = MX ? mxdata + static_cast<uint64_t>(off8) * 8 : nullptr;         \
-    uint8_t* mxs = MX ? mxscale + (off8 >> 2) : nullptr;                            \
-    uint16_t* cdst = MX ? nullptr : cache + static_cast<uint64_t>(off8) * 8;        \
-    if constexpr (gamma_in_smem<W, MX>()) {                                             \
+    float2 gs[4];                                                                   \
+    if constexpr (gamma_in_smem<W, MX>()) lds_gamma(my_gamma, gs);                  \
+    const float ss_ = group_sum<D / 8>(sum_sq8(acc));                               \
+    SCALE_STORE(acc, rsqrt_approx(fmaf(ss_, inv_d, eps)),                           \
+                (gamma_in_smem<W, MX>() ? gs : gm), off);                           \
+  } while (0)
+  // NB tokens from row `rb` of the stage: conv, their 1/rms together
+  // (head_rsqrt_batch), then scale and store each; the batch's NB row
+  // offsets are one vector load (rb is a multiple of NB)
+#define FAST_BATCH(rb)                                                              \
+  do {                                                                              \
+    float2 acc[NB][4];                                                              \
+    float ss[NB], rn[NB];                                                           \
+    _Pragma("unroll") for (int u = 0; u < NB; ++u) {                                \
+      const uint4 xr = *reinterpret_cast<const uint4*>(stage + ((rb) + u) * my_rs); \
+      conv_step<W>(tw, part, xr, acc[u]);                                           \
+      ss[u] = sum_sq8(acc[u]);                                                      \
+    }                                                                               \
+    head_rsqrt_batch<D / 8, NB>(ss, inv_d, eps, rn);                                \
+    uint32_t offs[NB];                                                              \
+    if constexpr (kVecOffsets) load_offsets<NB>(warp_off + sbase + (rb), offs);     \
+    _Pragma("unroll") for (int u = 0; u < NB; ++u) {                                \
+      if constexpr (!kVecOffsets) offs[u] = warp_off[sbase + (rb) + u];             \
       float2 gs[4];                                                                 \
-      lds_gamma(my_gamma, gs);                                                      \
-      norm_store<D, MX>(acc, gs, inv_d, eps, (pred), cdst, mxd, mxs);               \
-    } else {                                                                        \
-      norm_store<D, MX>(acc, gm, inv_d, eps, (pred), cdst, mxd, mxs);               \
+      if constexpr (gamma_in_smem<W, MX>()) lds_gamma(my_gamma, gs);                \
+      SCALE_STORE(acc[u], rn[u], (gamma_in_smem<W, MX>() ? gs : gm), active ? offs[u] : kNoRow); \
     }                                                                               \
   } while (0)
   // inactive lanes read column 0 (and never store): no predicated loads
@@ -682,29 +853,18 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
       // Where the unroll is shorter than a chunk, the tokens go in groups of
       // UF and a range's last, partial chunk skips the groups wholly past
       // its end (a short launch's ranges end in such a chunk).
-      constexpr int UF = fast_unroll<W, MX>();
+      constexpr int UF = fast_unroll<W, MX, LV>();
+      constexpr int NB = norm_batch<W, MX, LV, NBX>();
+      static_assert(UF % NB == 0, "an unrolled group is a whole number of batches");
       if constexpr (UF < R) {
         static_assert(R % UF == 0, "a chunk is a whole number of groups");
         for (int rb = 0; rb < rows; rb += UF) {
 #pragma unroll
-          for (int u = 0; u < UF; ++u) {
-            const int r = rb + u;
-            const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
-            float2 acc[4];
-            conv_step<W>(tw, win, xr, acc);
-            const uint32_t off8 = warp_off[sbase + r];
-            NORM_STORE(active && off8 != kNoRow);
-          }
+          for (int u0 = 0; u0 < UF; u0 += NB) FAST_BATCH(rb + u0);
         }
       } else {
-#pragma unroll fast_unroll<W, MX>()
-        for (int r = 0; r < R; ++r) {
-          const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
-          float2 acc[4];
-          conv_step<W>(tw, win, xr, acc);
-          const uint32_t off8 = warp_off[sbase + r];
-          NORM_STORE(active && off8 != kNoRow);
-        }
+#pragma unroll
+        for (int u0 = 0; u0 < R; u0 += NB) FAST_BATCH(u0);
       }
     } else {
       for (int r = 0; r < rows; ++r) {
@@ -717,9 +877,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
         }
         const uint4 xr = *reinterpret_cast<const uint4*>(stage + r * my_rs);
         float2 acc[4];
-        conv_step<W>(tw, win, xr, acc);
-        const uint32_t off8 = warp_off[sbase + r];
-        NORM_STORE(active && !skip && off8 != kNoRow);
+        conv_step<W>(tw, part, xr, acc);
+        NORM_STORE(active && !skip ? warp_off[sbase + r] : kNoRow);
       }
     }
     __syncwarp();
@@ -748,12 +907,14 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
     }
   }
 #undef NORM_STORE
+#undef SCALE_STORE
+#undef FAST_BATCH
 }
 
-template <int W, int D, int MINB, bool MX, bool LV>
+template <int W, int D, int MINB, bool MX, bool LV, int NBX = 0>
 __global__ void __launch_bounds__(prefill_threads<W, MX>(), MINB)
     prefill_tma_kernel(const StepParams P, const TmaGeom Gm) {
-  prefill_body<W, D, MX, LV>(P, Gm);
+  prefill_body<W, D, MX, LV, NBX>(P, Gm);
   // With the state-only dependency a CTA that never touched a state row has
   // not waited for the previous grid yet: it does before it exits, so this
   // grid's completion still implies its predecessor's.

@@ -347,6 +347,16 @@ int prefill_impl(
   if (ctas > by_tokens) ctas = by_tokens;
   if (ctas < 1) ctas = 1;
   G.ctas = static_cast<int>(ctas);
+  // a short bf16 launch (few chunks per CTA) takes the instance made for
+  // its compute-bound tail, when it is resident on the same terms
+  if (!mx && !uses_layout_variants(opts) &&
+      num_tokens <= static_cast<int64_t>(G.ctas) * R * SCONV_PREFILL_SHORT_CHUNKS) {
+    const TmaFn fs = sconv::pick_prefill_bf16_short(W, head_dim);
+    if (fs && smem_attr_set(reinterpret_cast<const void*>(fs), smem) &&
+        resident_per_sm(reinterpret_cast<const void*>(fs), static_cast<int>(block.x), smem,
+                        per_sm) >= occ)
+      fn = fs;
+  }
 #ifndef SCONV_PREFILL_SEQ_COST
 #define SCONV_PREFILL_SEQ_COST 16  // tokens a sequence start is worth when cutting ranges
 #endif
