@@ -68,7 +68,7 @@ def _check(b, got, ref):
 
 # ------------------------------------------------------------ per-head gamma
 
-@pytest.mark.parametrize("W,Hkv,D", [(4, 4, 128), (8, 3, 64), (2, 2, 256)])
+@pytest.mark.parametrize("W,Hkv,D", [(4, 4, 128), (3, 2, 64), (8, 3, 64), (2, 2, 256)])
 def test_per_head_gamma_prefill(W, Hkv, D):
     b = wl.make_prefill([300, 1, 0, 77, 9], Hkv=Hkv, D=D, W=W, seed=2800 + W, state="normal",
                         page_size=16, spare_pages=2)
@@ -137,7 +137,7 @@ def test_gamma_head_stride_rejected():
 
 # ------------------------------------------------------------ ring state
 
-@pytest.mark.parametrize("W", [2, 4, 8])
+@pytest.mark.parametrize("W", [2, 3, 4, 8])
 def test_ring_prefill(W):
     lengths = [0, 1, 2, 3, 9, 40, 700]
     b = wl.make_prefill(lengths, Hkv=4, D=128, W=W, seed=2840 + W, state="normal",

@@ -47,6 +47,31 @@ def test_single_8192_full():
     gu.full_parity(wl.single())
 
 
+def test_short_launch_instance_threshold_full():
+    """Around the token count where the host switches between the
+    short-launch bf16 instance (at most 8 chunks of 8 rows per persistent
+    CTA; 4-token head reductions) and the default one (2-token reductions):
+    both calls equal the oracle, and the rows they share are bitwise equal
+    (the batched reductions add the same lane sets in the same order)."""
+    import dataclasses
+    ctas = torch.cuda.get_device_properties(0).multi_processor_count * 2
+    Ts = ctas * 8 * 8  # largest single-sequence launch of the short instance
+    b = wl.make_prefill([Ts + 8], Hkv=2, D=128, W=4, seed=2190, state="normal",
+                        page_size=64, permute_pages=True)
+    short = dataclasses.replace(b, k=b.k[:Ts].clone(), v=b.v[:Ts].clone(),
+                                cu_seqlens=torch.tensor([0, Ts], dtype=torch.int32),
+                                slot_mapping=b.slot_mapping[:Ts].clone())
+    gu.full_parity(b)
+    gu.full_parity(short)
+    kl, vl, _ = gu.run_gpu_prefill(b)
+    ks, vs, _ = gu.run_gpu_prefill(short)
+    rows = b.slot_mapping[:Ts].numpy()
+    for a, c in ((kl, ks), (vl, vs)):
+        la = wl.bits(a.cpu()).reshape(-1, 2 * 128)[rows]
+        lc = wl.bits(c.cpu()).reshape(-1, 2 * 128)[rows]
+        assert np.array_equal(la, lc)
+
+
 @pytest.mark.parametrize("i", range(7))
 def test_partial_last_chunks_full(i):
     """Ranges ending in a partial chunk of every length 1..7 (one sequence,
