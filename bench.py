@@ -83,12 +83,38 @@ def algorithmic_bytes(tokens, seqs, W, Hkv, D, slot_bytes=8, mx=False, ring=Fals
     return tokens * per_token + seqs * per_seq + per_launch
 
 
+def strip_comments(src):
+    """C/C++ source without its comments, whitespace runs collapsed (string
+    and character literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash(kernel):
-    """Hash of the sources of `kernel` (a key of KERNEL_SOURCES)."""
+    """Hash of the code of `kernel`'s sources (a key of KERNEL_SOURCES),
+    comments and layout excluded: an edit to a comment keeps a profile."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

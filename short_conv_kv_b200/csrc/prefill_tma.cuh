@@ -26,16 +26,17 @@
 // released it) with chunk c-1+stages.  Loads in flight therefore do not
 // occupy registers: each CTA keeps up to a ring's worth of rows requested
 // while it computes.  (No separate producer warp: a 256-thread CTA may use
-// up to 255 registers per thread, which the W <= 8 register window needs.)
+// up to 255 registers per thread, which the W <= 8 carried partials need.)
 //
 // Consumers.  Consumer thread g owns 8 channels (16 bytes of a row) and walks
-// the rows in token order keeping the last W-1 rows in fp32 registers, as a
-// causal depthwise window.  Per token: conv (packed-fp32 FMAs), per-head sum of
-// squares (in-thread, then xor shuffles over D/8 lanes), rsqrt, gamma, round
-// to bf16, one 16-byte streaming store into the cache slot.  At a sequence
-// start the window is loaded from the sequence's conv_state and the new state
-// (the sequence's last W-1 raw rows) is written by the same thread over the
-// rows it has just read.
+// the rows in token order, carrying the causal depthwise conv in fp32
+// registers as W-1 partial sums (transposed form, conv_step).  Per token:
+// conv (packed-fp32 FMAs), per-head sum of squares (in-thread, then xor
+// shuffles over D/8 lanes, a few tokens at once in the fast path), rsqrt,
+// gamma, round to bf16 (or the MXFP8 block encoding), one streaming store
+// into the cache slot.  At a sequence start the partials are built from the
+// sequence's conv_state and the new state (the sequence's last W-1 raw rows)
+// is written by the same thread over the rows it has just read.
 #pragma once
 #include "common.cuh"
 #include "tma.cuh"
@@ -585,10 +586,10 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
   tb = max(ta, cut(blockIdx.x + 1));
   if (ta >= tb) return;
   // The CTA walks rows from first_row.  Rows first_row .. ta-1 (at most W-2,
-  // all in chunk 0) belong to the previous range: they only fill the
-  // window, and their stores are masked through the slot table.  A moved
-  // cut puts ta at position W-1 of its sequence (the window then holds
-  // rows 0 .. W-2 of it) or at a sequence start (whose window is loaded
+  // all in chunk 0) belong to the previous range: they only feed the conv's
+  // partials, and their stores are masked through the slot table.  A moved
+  // cut puts ta at position W-1 of its sequence (the partials then cover
+  // rows 0 .. W-2 of it) or at a sequence start (whose partials are built
   // from its state).  An empty range has requested nothing: its even range
   // is shorter than W-1 < R rows.
   const int seq0 = seq_of(first_row);
@@ -688,8 +689,8 @@ __device__ __forceinline__ void prefill_body(const StepParams& P, const TmaGeom&
     return true;
   };
 
-  // Enter sequence `i` at its first token: validate, load the old state into
-  // the window, write the new state.
+  // Enter sequence `i` at its first token: validate, build the conv's
+  // partials from the old state, write the new state.
   auto start_sequence = [&](int i) {
     int64_t si;
     skip = !check_sequence(i, si);
